@@ -1,0 +1,51 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check that
+the pins catch each one (CPU only; the planted mistakes never reach a GPU)."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in ln_oracle.c, replacement): each is a mistake someone could
+# plausibly make when writing LayerNorm and its hand-derived gradient.
+MUTANTS = [
+    ("unbiased_variance", "double var = sq / (double)C;",
+     "double var = sq / (double)(C - 1);"),
+    ("mean_divisor", "double m = sum / (double)C;",
+     "double m = sum / (double)(C + 1);"),
+    ("eps_outside_root", "1.0 / sqrt(var + eps)", "1.0 / (sqrt(var) + eps)"),
+    ("eps_dropped", "1.0 / sqrt(var + eps)", "1.0 / sqrt(var + 1e-300)"),
+    ("affine_swapped", "o[c] = xhat * weight[c] + bias[c];",
+     "o[c] = xhat * bias[c] + weight[c];"),
+    ("dinp_mean_term_dropped", "(g - mean_g - xhat * mean_gxhat)",
+     "(g - xhat * mean_gxhat)"),
+    ("dinp_xhat_term_dropped", "(g - mean_g - xhat * mean_gxhat)", "(g - mean_g)"),
+    ("dinp_sign_flipped", "(g - mean_g - xhat * mean_gxhat)",
+     "(g - mean_g + xhat * mean_gxhat)"),
+    ("dinp_rstd_dropped", "dx[c] = s * (", "dx[c] = ("),
+    ("g_without_weight", "double g = dy[c] * weight[c];", "double g = dy[c];"),
+    ("dweight_without_xhat", "dweight[c] += dy[c] * xhat;", "dweight[c] += dy[c];"),
+    ("xhat_divides_by_rstd", "double xhat = (x[c] - m) * s;",
+     "double xhat = (x[c] - m) / s;"),
+    ("dbias_times_weight", "dbias[c] += dy[c];", "dbias[c] += dy[c] * weight[c];"),
+    ("dweight_uses_g", "dweight[c] += dy[c] * xhat;", "dweight[c] += g * xhat;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert old in src, f"mutation site for {name} no longer in the oracle source"
+    mutant_src = os.path.join(tmp_path, f"{name}.c")
+    with open(mutant_src, "w") as f:
+        f.write(src.replace(old, new))
+    lib = oracle.compile_oracle(mutant_src, os.path.join(tmp_path, f"{name}.so"))
+    mutant = oracle.Oracle(library=lib, source=mutant_src)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, FloatingPointError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the mutant {name}"

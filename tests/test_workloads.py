@@ -1,0 +1,60 @@
+"""The seeded input generator (CPU only)."""
+import numpy as np
+
+from layernorm_fwd_bwd_b200 import workloads as wl
+
+
+def test_splitmix64_published_values():
+    # SplitMix64 with state seed + k*gamma; seed 0 first outputs as published
+    # with the algorithm (Steele, Lea, Flood 2014; Vigna's splitmix64.c).
+    z = np.uint64(0) + wl.GAMMA
+    assert int(wl.raw64(0, 0, np.array([0], np.uint64))[0]) == int(wl._finalise(np.array([z]))[0])
+    # seed 0: the first three SplitMix64 outputs
+    first = [int(v) for v in wl.raw64(0, 0, np.arange(3, dtype=np.uint64))]
+    assert first == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_rows_subset_matches_full():
+    work = wl.Workload("t", wl.BF16, 300, 40, 7, dout_sigma=0.02)
+    full = wl.generate(work)
+    rows = np.array([0, 5, 17, 299])
+    part = wl.generate(work, rows)
+    assert np.array_equal(full.inp[rows], part.inp)
+    assert np.array_equal(full.dout[rows], part.dout)
+    assert np.array_equal(full.weight, part.weight)
+
+
+def test_bf16_rounding_is_nearest_even():
+    one = 1.0
+    ulp = 2.0 ** -7
+    v = np.array([one + ulp / 2, one + 1.5 * ulp, one + ulp / 2 + 1e-12, -3.0,
+                  0.0, 1e-3])
+    bits = wl.round_bf16_bits(v)
+    back = wl.bf16_bits_to_f64(bits)
+    assert back[0] == 1.0                 # tie -> even (down)
+    assert back[1] == one + 2 * ulp       # tie -> even (up)
+    assert back[2] == one + ulp           # above the tie -> up
+    assert back[3] == -3.0 and back[4] == 0.0
+    assert abs(back[5] - 1e-3) <= 1e-3 * 2.0 ** -8
+
+
+def test_distributions():
+    b = wl.generate(wl.WORKLOADS["gpt2_124m_bf16"], rows=np.arange(512))
+    x, dy = b.f64("inp"), b.f64("dout")
+    assert abs(x.mean()) < 0.01 and abs(x.std() - 1) < 0.01
+    assert abs(dy.std() - 0.02) < 0.001
+    assert abs(b.f64("weight").mean() - 1) < 0.02
+    s = wl.generate(wl.WORKLOADS["stress_fp32_65536x768"], rows=np.arange(0, 1000))
+    xs = s.f64("inp")
+    const = np.arange(1000) % 100 == 0
+    assert np.all(xs[const].std(axis=1) == 0)
+    assert np.all(np.abs(xs[~const].std(axis=1) - 0.01) < 0.002)
+    assert abs(xs.mean() - 100) < 0.01
+
+
+def test_compulsory_bytes():
+    w = wl.WORKLOADS["gpt2_124m_bf16"]
+    assert w.fwd_bytes() == 201_853_952
+    assert w.bwd_bytes() == 302_521_856
+    assert wl.WORKLOADS["stress_fp32_65536x768"].fwd_bytes() + \
+        wl.WORKLOADS["stress_fp32_65536x768"].bwd_bytes() == 1_007_696_896
