@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark: LayerNorm forward + analytical backward on B200 (sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step = one ``ln_forward`` and one ``ln_backward`` call (every step of the
+hot path: row statistics, normalise + affine, row gradient sums, dinp, column
+partials, fixed-order column finalise) over one batch of the workload
+(default: GPT-2 124M LayerNorm, bf16 activations, N = 65536 rows, C = 768).
+
+Metric: compulsory HBM bytes of forward + backward per second (GB/s), with
+rows/s and the fraction of the measured HBM copy bandwidth beside it.
+Compulsory bytes: forward 2*N*C*s + 8N + 2*C*s, backward 3*N*C*s + 8N + C*s
++ 8C (s = bytes per activation element).
+
+Timing: inputs resident in HBM before the timed region; W untimed warm-up
+steps; K timed steps bracketed by a barrier and a device synchronise on both
+sides, timed with CUDA events on the launching stream; max over ranks.  L2:
+four buffer sets rotate (each 4*N*C*s bytes, 403 MB for the default
+workload), and a step's backward reads a set that its forward did not touch,
+so no step re-reads an input from the 126 MB L2.
+
+With N > 1 (torchrun, one rank per GPU) every rank processes its own batch
+(weak scaling, data-parallel row shards); the path has no exchange step.
+
+``--impl reference`` times the CPU oracle (double precision, the parity
+reference) on host cores on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LayerNorm fwd+bwd GB/s and rows/s at 1 B200; % of HBM roofline"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+SETS = 4
+KERNEL_SOURCES = [os.path.join(ROOT, "layernorm_fwd_bwd_b200", "csrc", f)
+                  for f in ("ln_kernels.cuh", "ln_api.cu")]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "ln_backward_gpt2_124m_bf16.md")
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--workload", default="gpt2_124m_bf16")
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=0,
+                   help="end-to-end steps (0: K/500, at least 8)")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--sets", type=int, default=SETS,
+                   help="rotating buffer sets (>= 2 so a step's backward never "
+                        "reads what its forward just read)")
+    return p.parse_args()
+
+
+def source_sha256() -> str:
+    h = hashlib.sha256()
+    for path in KERNEL_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per ln_backward call from the committed ncu summary, or None
+    when it is missing or was taken on different kernel sources."""
+    try:
+        text = open(TRAFFIC_PROFILE).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_call:\s*(\d+)", text)
+    s = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not s or s.group(1) != source_sha256():
+        return None
+    return int(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        self.file.seek(0)
+        rows = []
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        inside = [r for r in rows if t0 - 0.25 <= r[0] <= t1 + 0.25]
+        if not inside:
+            # region shorter than the sampling period: nearest sample(s)
+            inside = sorted(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))[:2]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"],
+                    "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[k] for r in inside for k in range(4)
+                          if r[3][k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# --------------------------------------------------------------------- ours
+
+def run_ours(args, world: int, rank: int, local: int):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from layernorm_fwd_bwd_b200 import ln
+    from layernorm_fwd_bwd_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    N, C = w.N, w.C
+    tdt = torch.float32 if w.dtype == wl.F32 else torch.bfloat16
+    dcode = ln.LN_F32 if w.dtype == wl.F32 else ln.LN_BF16
+    batch = wl.generate(w)
+
+    def host_tensor(a):
+        if w.dtype == wl.F32:
+            return torch.from_numpy(np.ascontiguousarray(a, np.float32))
+        return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(
+            torch.bfloat16)
+
+    h_inp, h_dout = host_tensor(batch.inp), host_tensor(batch.dout)
+    h_w, h_b = host_tensor(batch.weight), host_tensor(batch.bias)
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        weight, bias = h_w.to(dev), h_b.to(dev)
+        dweight = torch.empty(C, device=dev)
+        dbias = torch.empty(C, device=dev)
+        sets = []
+        nsets = max(2, args.sets)
+        for _ in range(nsets):
+            sets.append(dict(inp=h_inp.to(dev), dout=h_dout.to(dev),
+                             out=torch.empty(N, C, dtype=tdt, device=dev),
+                             dinp=torch.empty(N, C, dtype=tdt, device=dev),
+                             mean=torch.empty(N, device=dev),
+                             rstd=torch.empty(N, device=dev)))
+    stream.synchronize()
+    eps = batch.eps
+    fargs = [(s["out"].data_ptr(), s["mean"].data_ptr(), s["rstd"].data_ptr(),
+              s["inp"].data_ptr(), weight.data_ptr(), bias.data_ptr(), N, C, eps,
+              dcode, sp) for s in sets]
+    bargs = [(s["dinp"].data_ptr(), dweight.data_ptr(), dbias.data_ptr(),
+              s["dout"].data_ptr(), s["inp"].data_ptr(), weight.data_ptr(),
+              s["mean"].data_ptr(), s["rstd"].data_ptr(), N, C, dcode, sp)
+             for s in sets]
+    fwd, bwd = ln.raw_forward, ln.raw_backward
+
+    def check(rc):
+        if rc != 0:
+            raise ln.LNError(rc)
+
+    for k in range(nsets):                      # statistics for every set
+        check(fwd(*fargs[k]))
+
+    def step(i, ev=None):
+        a, b = i % nsets, (i + nsets // 2) % nsets
+        if ev is not None:
+            ev[0].record(stream)
+        check(fwd(*fargs[a]))
+        if ev is not None:
+            ev[1].record(stream)
+        check(bwd(*bargs[b]))
+        if ev is not None:
+            ev[2].record(stream)
+
+    K, W = args.steps, args.warmup
+    sampler = ClockSampler(local) if rank == 0 else None
+    for i in range(W):
+        step(i)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ln.launch_count()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(K):
+        step(W + i, events[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    launches = ln.launch_count() - launches0
+    if sampler is not None:
+        sampler.stop()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in events)
+    bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in events)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = None if args.no_e2e else run_e2e(args, torch, ln, stream, dev, h_inp, h_dout,
+                                           h_w, h_b, N, C, tdt, dcode, eps, world)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    fb, bb = w.fwd_bytes(), w.bwd_bytes()
+    step_s = total_ms / 1e3 / K
+    value = world * (fb + bb) / step_s / 1e9
+    peak, peak_kind = hbm_peak()
+    bwd_gbs = bb / (bwd_ms / 1e3) / 1e9
+    fwd_gbs = fb / (fwd_ms / 1e3) / 1e9
+    clocks = sampler.summary(t0, t1) if sampler else None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(total_ms / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded SplitMix64/Box-Muller, workload distributions)",
+        "config": {"workload": w.name, "description": w.description, "N": N, "C": C,
+                   "activations": w.dtype, "stats_and_param_grads": "f32",
+                   "eps": eps, "rows_per_gpu": N, "parallelism": f"dp{world} (row shards)",
+                   "l2": f"{nsets} rotating buffer sets; each step's backward reads a set "
+                         "its forward did not touch; inputs never re-read from L2"},
+        "rows_per_s": round(world * N / step_s, 1),
+        "pct_hbm_measured": round(value / world / peak * 100, 2) if peak_kind == "measured" else None,
+        "pct_hbm_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS * 100, 2),
+        "fwd": {"us": round(fwd_ms * 1e3, 3), "GB_s": round(fwd_gbs, 1),
+                "bytes": fb},
+        "bwd": {"us": round(bwd_ms * 1e3, 3), "GB_s": round(bwd_gbs, 1),
+                "bytes": bb},
+        "roofline": {"bound": "hbm", "kernel": "ln_backward (row pass + column finalise)",
+                     "achieved": round(bwd_gbs, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(bwd_gbs / peak, 4),
+                     "traffic": profiled_traffic()},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    line["cpu_baseline"] = (None if (world > 1 or args.no_cpu_baseline)
+                            else cpu_baseline(w, args.cpu_seconds))
+    return line
+
+
+def run_e2e(args, torch, ln, stream, dev, h_inp, h_dout, h_w, h_b, N, C, tdt, dcode,
+            eps, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory, runs forward and backward, and reads
+    every result back into pinned host memory."""
+    steps = args.e2e_steps or max(8, args.steps // 500)
+    pin = {k: v.pin_memory() for k, v in
+           dict(inp=h_inp, dout=h_dout, w=h_w, b=h_b).items()}
+    hout = {k: torch.empty(shape, dtype=dt).pin_memory() for k, (shape, dt) in dict(
+        out=((N, C), tdt), dinp=((N, C), tdt), mean=((N,), torch.float32),
+        rstd=((N,), torch.float32), dw=((C,), torch.float32),
+        db=((C,), torch.float32)).items()}
+    with torch.cuda.stream(stream):
+        d = dict(inp=torch.empty(N, C, dtype=tdt, device=dev),
+                 dout=torch.empty(N, C, dtype=tdt, device=dev),
+                 w=torch.empty(C, dtype=tdt, device=dev),
+                 b=torch.empty(C, dtype=tdt, device=dev),
+                 out=torch.empty(N, C, dtype=tdt, device=dev),
+                 dinp=torch.empty(N, C, dtype=tdt, device=dev),
+                 mean=torch.empty(N, device=dev), rstd=torch.empty(N, device=dev),
+                 dw=torch.empty(C, device=dev), db=torch.empty(C, device=dev))
+
+    def one():
+        with torch.cuda.stream(stream):
+            for k in ("inp", "dout", "w", "b"):
+                d[k].copy_(pin[k], non_blocking=True)
+            ln.ln_forward(d["out"], d["mean"], d["rstd"], d["inp"], d["w"], d["b"], N, C,
+                          eps, dcode, stream)
+            ln.ln_backward(d["dinp"], d["dw"], d["db"], d["dout"], d["inp"], d["w"],
+                           d["mean"], d["rstd"], N, C, dcode, stream)
+            for k in hout:
+                hout[k].copy_(d[k], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    from layernorm_fwd_bwd_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = sum(v.numel() * v.element_size() for v in hout.values())
+    step_s = ms / 1e3 / steps
+    return {"value": round(world * (w.fwd_bytes() + w.bwd_bytes()) / step_s / 1e9, 2),
+            "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "ms_per_step": round(ms / steps, 4)}
+
+
+# ----------------------------------------------------------------- oracle
+
+def _oracle_rate(w, rows_sample: int, seconds: float):
+    """Time the CPU oracle (as it stands) on a row sample: forward then
+    backward.  Returns (GB/s of compulsory bytes, seconds per pass, passes)."""
+    import numpy as np
+
+    import oracle
+    from layernorm_fwd_bwd_b200 import workloads as wl
+    rows = np.arange(rows_sample, dtype=np.int64)
+    b = wl.generate(w, rows=rows)
+    x, dy = b.f64("inp"), b.f64("dout")
+    wt, bs = b.f64("weight"), b.f64("bias")
+    orc = oracle.default()
+    times = []
+    t_end = time.perf_counter() + seconds
+    while True:
+        t = time.perf_counter()
+        _, m, r = orc.forward(x, wt, bs, b.eps)
+        orc.backward(dy, x, wt, m, r)
+        times.append(time.perf_counter() - t)
+        if time.perf_counter() >= t_end and len(times) >= 1:
+            break
+    s = w.elem_bytes
+    n = rows_sample
+    byts = (2 * n * w.C * s + 8 * n + 2 * w.C * s) + (3 * n * w.C * s + 8 * n + w.C * s + 8 * w.C)
+    per = statistics.median(times)
+    return byts / per / 1e9, per, len(times)
+
+
+def cpu_baseline(w, seconds: float) -> dict:
+    rows = min(w.N, 16384)
+    gbs, per, reps = _oracle_rate(w, rows, seconds)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {w.N} rows of {w.name}, forward+backward in "
+                      f"double, median of {reps} passes ({per:.3f} s each), "
+                      "single thread"}
+
+
+def run_reference(args, world: int, rank: int):
+    """The CPU oracle timed as the reference arm: each step is forward +
+    backward over a bounded row sample of the same workload."""
+    if rank != 0:
+        return None
+    from layernorm_fwd_bwd_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    # calibrate: rows per second of the oracle on a small sample
+    _, per, _ = _oracle_rate(w, 512, 0.0)
+    rows_per_s = 512 / per
+    budget = 150.0
+    rows = int(max(1, min(w.N, rows_per_s * budget / max(1, args.steps + args.warmup))))
+    import numpy as np
+
+    import oracle
+    b = wl.generate(w, rows=np.arange(rows, dtype=np.int64))
+    x, dy = b.f64("inp"), b.f64("dout")
+    wt, bs = b.f64("weight"), b.f64("bias")
+    orc = oracle.default()
+    for _ in range(args.warmup):
+        _, m, r = orc.forward(x, wt, bs, b.eps)
+        orc.backward(dy, x, wt, m, r)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        _, m, r = orc.forward(x, wt, bs, b.eps)
+        orc.backward(dy, x, wt, m, r)
+    el = time.perf_counter() - t
+    s = w.elem_bytes
+    byts = (2 * rows * w.C * s + 8 * rows + 2 * w.C * s) + \
+        (3 * rows * w.C * s + 8 * rows + w.C * s + 8 * w.C)
+    value = byts * args.steps / el / 1e9
+    sample = (f"first {rows} of {w.N} rows of {w.name} per step, forward+backward in "
+              "double, single thread")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded SplitMix64/Box-Muller, workload distributions)",
+        "config": {"workload": w.name, "description": w.description, "N": w.N, "C": w.C,
+                   "activations": w.dtype, "rows_per_step_sample": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE",
+              file=sys.stderr)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+    if line is not None and rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,131 @@
+/*
+ * ln.h -- C ABI of libln.so: LayerNorm forward and analytical backward on an
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation.  "llm.c's Origin and the Future of LLM Compilers" (CUDA MODE
+ * talk page), chapter "Deconstructing PyTorch Abstractions and Setting
+ * Reference Baselines", describes LayerNorm forward and backward written over
+ * bare float arrays with no tensor abstraction; "llm.c: Large Language Model
+ * Training in Pure C/CUDA Without Dependencies", features "Tensor Memory
+ * Layout" (flat 1-D row-major arrays, explicit stride arithmetic) and "Exact
+ * Analytical Backward Pass" (hand-derived LayerNorm gradients).  The pages do
+ * not print the equations; this library computes the textbook definition:
+ *
+ *   mean[r] = (1/C) sum_c x[r,c]
+ *   rstd[r] = 1 / sqrt((1/C) sum_c (x[r,c] - mean[r])^2 + eps)
+ *   out     = (x - mean[r]) * rstd[r] * weight[c] + bias[c]
+ *
+ *   xhat    = (x - mean[r]) * rstd[r],   g = dout * weight[c]
+ *   dinp    = rstd[r] * (g - (1/C) sum_c g - xhat * (1/C) sum_c g * xhat)
+ *   dweight = sum over all N rows of dout * xhat
+ *   dbias   = sum over all N rows of dout
+ *
+ * Layout.  Activations (inp, out, dout, dinp) are flat row-major [N * C]
+ * arrays: row r starts at element r * C.  weight, bias, dweight and dbias hold
+ * C elements, mean and rstd hold N.  All pointers are DEVICE pointers of the
+ * current CUDA device, owned by the caller; the library never frees them.
+ *
+ * Types.  `dtype` (LN_F32 or LN_BF16) is the element type of inp, out, dout,
+ * dinp, weight and bias.  mean, rstd, dweight and dbias are always fp32.
+ * Arithmetic is fp32 in registers; bf16 results are rounded to nearest-even.
+ *
+ * Semantics shared by both calls.
+ *   - Asynchronous on `stream` (NULL: the legacy default stream); no host
+ *     synchronisation; the library creates no streams of its own.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Results are deterministic: the same inputs give bitwise-identical
+ *     outputs on every call (no floating-point atomics).
+ *   - Any alignment is accepted.  Fully 16-byte-aligned arrays with C * size
+ *     a multiple of 16 bytes take the vectorised path; others a scalar path.
+ *   - Errors are returned as an ln_status value; nothing is launched when
+ *     validation fails, and no kernel asserts or traps.
+ *   - 1 <= C <= LN_MAX_C; 0 <= N <= LN_MAX_N; N * C <= LN_MAX_ELEMS.
+ *     N == 0 launches nothing in the forward; in the backward it only
+ *     zero-fills dweight and dbias (pointers other than dweight and dbias
+ *     may then be NULL).
+ */
+#ifndef LN_H
+#define LN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that C callers need no CUDA
+ * header. */
+struct CUstream_st;
+typedef struct CUstream_st *ln_stream_t;
+
+#define LN_MAX_C ((int64_t)1 << 24)
+#define LN_MAX_N ((int64_t)1 << 40)
+#define LN_MAX_ELEMS ((int64_t)1 << 50)   /* bound on N * C */
+
+typedef enum {
+    LN_F32 = 0,   /* IEEE binary32 */
+    LN_BF16 = 1   /* bfloat16 (8 significant bits, binary32 exponent range) */
+} ln_dtype;
+
+typedef enum {
+    LN_OK = 0,
+    LN_ERR_NULL = 1,       /* a required pointer is NULL */
+    LN_ERR_SHAPE = 2,      /* N < 0, N > LN_MAX_N, C < 1, C > LN_MAX_C or
+                              N * C > LN_MAX_ELEMS */
+    LN_ERR_DTYPE = 3,      /* dtype is not LN_F32 or LN_BF16 */
+    LN_ERR_EPS = 4,        /* eps is not finite, or not > 0 */
+    LN_ERR_WORKSPACE = 5,  /* the backward's workspace could not be allocated */
+    LN_ERR_CUDA = 6        /* a CUDA runtime call or launch failed */
+} ln_status;
+
+/*
+ * LayerNorm forward over N rows of C channels.
+ *   out   [N*C] dtype, written      normalised, scaled and shifted rows
+ *   mean  [N]   fp32,  written      per-row mean
+ *   rstd  [N]   fp32,  written      per-row 1/sqrt(var + eps), var biased (1/C)
+ *   inp   [N*C] dtype, read
+ *   weight, bias [C] dtype, read
+ *   eps   finite, > 0 (1e-5 in GPT-2)
+ * out must not overlap inp.  Returns LN_OK or an ln_status error.
+ */
+int ln_forward(void *out, float *mean, float *rstd, const void *inp,
+               const void *weight, const void *bias, int64_t N, int64_t C,
+               float eps, int dtype, ln_stream_t stream);
+
+/*
+ * LayerNorm backward for the loss gradient dout, given the statistics that
+ * ln_forward saved for the same inp.
+ *   dinp    [N*C] dtype, written    gradient w.r.t. inp
+ *   dweight [C]   fp32,  written    sum over rows of dout * xhat
+ *   dbias   [C]   fp32,  written    sum over rows of dout
+ *   dout    [N*C] dtype, read
+ *   inp     [N*C] dtype, read
+ *   weight  [C]   dtype, read
+ *   mean, rstd [N] fp32, read
+ * The column sums are formed in two stages with a fixed summation order:
+ * per-block partial sums into a library-owned workspace drawn, stream-ordered,
+ * from a per-device memory pool (returned to the pool on `stream` after use),
+ * then one fixed-order sum of the partials.  dinp must not overlap dout or
+ * inp.  Returns LN_OK or an ln_status error (LN_ERR_WORKSPACE when the pool
+ * cannot supply the workspace).
+ */
+int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
+                const void *inp, const void *weight, const float *mean,
+                const float *rstd, int64_t N, int64_t C, int dtype,
+                ln_stream_t stream);
+
+/* Static description of an ln_status value (never NULL). */
+const char *ln_status_string(int status);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams).  For accounting in benchmarks and tests. */
+uint64_t ln_launch_count(void);
+
+/* Library ABI version: 1. */
+int ln_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LN_H */

@@ -1,0 +1,403 @@
+// ln_api.cu -- C ABI of libln.so (declared in include/ln.h): argument
+// validation, kernel selection, launch geometry and the backward's workspace.
+//
+// Geometry.  Every kernel runs on a persistent grid of (SM count) x (resident
+// blocks per SM, from the occupancy calculator for the exact block size and
+// shared memory), capped by the number of rows.  Row ownership:
+//   C * sizeof(T) a multiple of 16 and all activation/parameter arrays
+//   16-byte aligned  -> vectorised kernels:
+//       C / E <= 32 * Vmax      one warp per row, 8 rows per 256-thread block,
+//                               V = ceil(C / E / 32) vectors per lane;
+//       C / E <= 32 * 32 * 4    W = 2..32 warps per row (2..16 in the backward),
+//                               4 vectors per thread;
+//   otherwise                -> scalar kernels (any alignment, any C).
+// where E = 16 / sizeof(T) elements per vector.
+//
+// Workspace.  The backward needs G * 2C fp32 partial sums (G = its grid).
+// They are drawn stream-ordered from a memory pool that the library creates
+// once per device (release threshold: never), and handed back on the same
+// stream right after the finalise kernel, so calls on different streams never
+// share a buffer and steady-state calls reuse pool memory without a
+// cudaMalloc.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/ln.h"
+#include "ln_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kRowsPerBlockW1 = 8;       // row groups per block, one warp per row
+constexpr int kMaxVecPerLaneFwd = 8;
+constexpr int kMaxVecPerLaneBwd = 8;
+constexpr int kMultiWarpVec = 4;         // vectors per thread with W > 1
+constexpr size_t kMaxWorkspaceBytes = size_t(256) << 20;
+
+std::atomic<uint64_t> g_launches{0};
+
+struct DeviceState {
+    std::once_flag once;
+    int sms = 0;
+    int max_smem_optin = 0;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t init_error = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+
+cudaError_t device_state(int dev, DeviceState **out) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    DeviceState &d = g_dev[dev];
+    std::call_once(d.once, [&]() {
+        cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&d.max_smem_optin,
+                                       cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            e = cudaMemPoolCreate(&d.pool, &props);
+        }
+        if (e == cudaSuccess) {
+            uint64_t keep = UINT64_MAX;
+            e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        d.init_error = e;
+    });
+    *out = &d;
+    return d.init_error;
+}
+
+// Occupancy (resident blocks per SM) per kernel, device and dynamic shared
+// memory size, computed once.
+struct OccKey {
+    const void *fn;
+    int dev;
+    int threads;
+    size_t smem;
+    bool operator==(const OccKey &o) const {
+        return fn == o.fn && dev == o.dev && threads == o.threads && smem == o.smem;
+    }
+};
+struct OccHash {
+    size_t operator()(const OccKey &k) const {
+        return std::hash<const void *>()(k.fn) ^ (size_t(k.dev) << 1) ^
+               (size_t(k.threads) << 8) ^ (k.smem << 20);
+    }
+};
+std::mutex g_occ_mu;
+std::unordered_map<OccKey, int, OccHash> g_occ;
+
+template <typename K>
+cudaError_t blocks_per_sm(K kernel, int dev, int threads, size_t smem, int *occ) {
+    const OccKey key{reinterpret_cast<const void *>(kernel), dev, threads, smem};
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        auto it = g_occ.find(key);
+        if (it != g_occ.end()) {
+            *occ = it->second;
+            return cudaSuccess;
+        }
+    }
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+    int n = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    g_occ[key] = n;
+    *occ = n;
+    return cudaSuccess;
+}
+
+template <typename K, typename... Args>
+cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
+                   bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? LN_OK : LN_ERR_CUDA; }
+
+// ------------------------------------------------------------------ forward
+
+struct FwdArgs {
+    void *out;
+    float *mean;
+    float *rstd;
+    const void *inp;
+    const void *weight;
+    const void *bias;
+    int64_t N;
+    int C;
+    float inv_C;
+    float eps;
+    cudaStream_t stream;
+    int dev;
+    int sms;
+};
+
+template <typename T, int V, int W, int GROUPS>
+cudaError_t fwd_vec(const FwdArgs &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    auto kern = lnk::ln_fwd_vec_kernel<T, V, W, GROUPS>;
+    const int threads = 32 * W * GROUPS;
+    const int nvec = a.C / E;
+    const size_t smem = size_t(2) * nvec * 16 + (W > 1 ? 2 * W * sizeof(float) : 0);
+    int occ = 0;
+    cudaError_t e = blocks_per_sm(kern, a.dev, threads, smem, &occ);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(ceil_div(a.N, GROUPS), int64_t(a.sms) * occ);
+    return launch(kern, (int)grid, threads, smem, a.stream, false,
+                  static_cast<T *>(a.out), a.mean, a.rstd, static_cast<const T *>(a.inp),
+                  static_cast<const T *>(a.weight), static_cast<const T *>(a.bias), a.N,
+                  a.C, a.inv_C, a.eps);
+}
+
+template <typename T, bool BLOCK_ROW>
+cudaError_t fwd_scalar(const FwdArgs &a) {
+    auto kern = lnk::ln_fwd_scalar_kernel<T, BLOCK_ROW>;
+    const int threads = BLOCK_ROW ? (a.C > 4096 ? 512 : 256) : 256;
+    const int groups = BLOCK_ROW ? 1 : threads / 32;
+    int occ = 0;
+    cudaError_t e = blocks_per_sm(kern, a.dev, threads, 0, &occ);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(ceil_div(a.N, groups), int64_t(a.sms) * occ);
+    return launch(kern, (int)grid, threads, 0, a.stream, false, static_cast<T *>(a.out),
+                  a.mean, a.rstd, static_cast<const T *>(a.inp),
+                  static_cast<const T *>(a.weight), static_cast<const T *>(a.bias), a.N,
+                  a.C, a.inv_C, a.eps);
+}
+
+template <typename T>
+cudaError_t fwd_dispatch(const FwdArgs &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.out) &&
+                        aligned16(a.inp) && aligned16(a.weight) && aligned16(a.bias);
+    if (vec_ok) {
+        const int nvec = a.C / E;
+        if (nvec <= 32 * kMaxVecPerLaneFwd) {
+            switch ((nvec + 31) / 32) {
+                case 1: return fwd_vec<T, 1, 1, kRowsPerBlockW1>(a);
+                case 2: return fwd_vec<T, 2, 1, kRowsPerBlockW1>(a);
+                case 3: return fwd_vec<T, 3, 1, kRowsPerBlockW1>(a);
+                case 4: return fwd_vec<T, 4, 1, kRowsPerBlockW1>(a);
+                case 5: return fwd_vec<T, 5, 1, kRowsPerBlockW1>(a);
+                case 6: return fwd_vec<T, 6, 1, kRowsPerBlockW1>(a);
+                case 7: return fwd_vec<T, 7, 1, kRowsPerBlockW1>(a);
+                default: return fwd_vec<T, 8, 1, kRowsPerBlockW1>(a);
+            }
+        }
+        const int per_warp = 32 * kMultiWarpVec;
+        if (nvec <= 2 * per_warp) return fwd_vec<T, kMultiWarpVec, 2, 1>(a);
+        if (nvec <= 4 * per_warp) return fwd_vec<T, kMultiWarpVec, 4, 1>(a);
+        if (nvec <= 8 * per_warp) return fwd_vec<T, kMultiWarpVec, 8, 1>(a);
+        if (nvec <= 16 * per_warp) return fwd_vec<T, kMultiWarpVec, 16, 1>(a);
+        if (nvec <= 32 * per_warp) return fwd_vec<T, kMultiWarpVec, 32, 1>(a);
+    }
+    if (a.C <= 1024) return fwd_scalar<T, false>(a);
+    return fwd_scalar<T, true>(a);
+}
+
+// ----------------------------------------------------------------- backward
+
+struct BwdArgs {
+    void *dinp;
+    float *dweight;
+    float *dbias;
+    const void *dout;
+    const void *inp;
+    const void *weight;
+    const float *mean;
+    const float *rstd;
+    int64_t N;
+    int C;
+    float inv_C;
+    cudaStream_t stream;
+    int dev;
+    int sms;
+    cudaMemPool_t pool;
+};
+
+// Runs the row kernel on G blocks of `rows_per_block` consecutive rows, then
+// the fixed-order column finalise (programmatic dependent launch).
+template <typename T, typename K>
+int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule) {
+    int occ = 0;
+    if (blocks_per_sm(kern, a.dev, threads, smem, &occ) != cudaSuccess) return LN_ERR_CUDA;
+    int64_t G = std::min<int64_t>(int64_t(a.sms) * occ, ceil_div(a.N, rows_granule));
+    // keep the partial sums within kMaxWorkspaceBytes (matters only for very
+    // wide rows, where fewer, longer-running blocks are the price)
+    G = std::min<int64_t>(G, int64_t(kMaxWorkspaceBytes / (size_t(a.C) * 2 * sizeof(float))));
+    G = std::max<int64_t>(G, 1);
+    const int64_t rows_per_block = ceil_div(a.N, G);
+    G = ceil_div(a.N, rows_per_block);
+
+    float *partial = nullptr;
+    const size_t ws_bytes = size_t(G) * 2 * size_t(a.C) * sizeof(float);
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), ws_bytes, a.pool,
+                                a.stream) != cudaSuccess) {
+        cudaGetLastError();   // clear the non-sticky allocation error
+        return LN_ERR_WORKSPACE;
+    }
+    cudaError_t e = launch(kern, (int)G, threads, smem, a.stream, false,
+                           static_cast<T *>(a.dinp), partial,
+                           static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                           static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C,
+                           a.inv_C, rows_per_block);
+    if (e == cudaSuccess) {
+        const int cblocks = (int)ceil_div(2 * int64_t(a.C), 32);
+        e = launch(lnk::ln_colsum_kernel, cblocks, 256, 0, a.stream, true, a.dweight,
+                   a.dbias, static_cast<const float *>(partial), (int)G, a.C);
+    }
+    const cudaError_t ef = cudaFreeAsync(partial, a.stream);
+    if (e == cudaSuccess) e = ef;
+    return status_of(e);
+}
+
+template <typename T, int V, int W, int GROUPS>
+int bwd_vec(const BwdArgs &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    const int threads = 32 * W * GROUPS;
+    const int nvec = a.C / E;
+    const size_t smem = size_t(nvec) * 16 + (GROUPS > 1 ? 2 * size_t(a.C) * 4 : 0) +
+                        (W > 1 ? 4 * W * sizeof(float) : 0);
+    return bwd_run<T>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>, threads, smem, GROUPS);
+}
+
+template <typename T>
+int bwd_scalar(const BwdArgs &a) {
+    int threads = (int)std::min<int64_t>(512, ceil_div(a.C, 32) * 32);
+    return bwd_run<T>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1);
+}
+
+template <typename T>
+int bwd_dispatch(const BwdArgs &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.dinp) &&
+                        aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
+    if (vec_ok) {
+        const int nvec = a.C / E;
+        if (nvec <= 32 * kMaxVecPerLaneBwd) {
+            switch ((nvec + 31) / 32) {
+                case 1: return bwd_vec<T, 1, 1, kRowsPerBlockW1>(a);
+                case 2: return bwd_vec<T, 2, 1, kRowsPerBlockW1>(a);
+                case 3: return bwd_vec<T, 3, 1, kRowsPerBlockW1>(a);
+                case 4: return bwd_vec<T, 4, 1, kRowsPerBlockW1>(a);
+                case 5: return bwd_vec<T, 5, 1, kRowsPerBlockW1>(a);
+                case 6: return bwd_vec<T, 6, 1, kRowsPerBlockW1>(a);
+                case 7: return bwd_vec<T, 7, 1, kRowsPerBlockW1>(a);
+                default: return bwd_vec<T, 8, 1, kRowsPerBlockW1>(a);
+            }
+        }
+        const int per_warp = 32 * kMultiWarpVec;
+        if (nvec <= 2 * per_warp) return bwd_vec<T, kMultiWarpVec, 2, 1>(a);
+        if (nvec <= 4 * per_warp) return bwd_vec<T, kMultiWarpVec, 4, 1>(a);
+        if (nvec <= 8 * per_warp) return bwd_vec<T, kMultiWarpVec, 8, 1>(a);
+        if (nvec <= 16 * per_warp) return bwd_vec<T, kMultiWarpVec, 16, 1>(a);
+        // 1024-thread blocks would cap registers at 64 and spill the column
+        // accumulators: wider rows take the scalar path.
+    }
+    return bwd_scalar<T>(a);
+}
+
+int current_device(int *dev, DeviceState **ds) {
+    if (cudaGetDevice(dev) != cudaSuccess) return LN_ERR_CUDA;
+    if (device_state(*dev, ds) != cudaSuccess) return LN_ERR_CUDA;
+    return LN_OK;
+}
+
+int check_shape(int64_t N, int64_t C) {
+    if (N < 0 || N > LN_MAX_N || C < 1 || C > LN_MAX_C) return LN_ERR_SHAPE;
+    if (N > LN_MAX_ELEMS / C) return LN_ERR_SHAPE;
+    return LN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ln_forward(void *out, float *mean, float *rstd, const void *inp, const void *weight,
+               const void *bias, int64_t N, int64_t C, float eps, int dtype,
+               ln_stream_t stream) {
+    if (int st = check_shape(N, C)) return st;
+    if (dtype != LN_F32 && dtype != LN_BF16) return LN_ERR_DTYPE;
+    if (!std::isfinite(eps) || !(eps > 0.f)) return LN_ERR_EPS;
+    if (N == 0) return LN_OK;
+    if (!out || !mean || !rstd || !inp || !weight || !bias) return LN_ERR_NULL;
+    int dev = 0;
+    DeviceState *ds = nullptr;
+    if (int st = current_device(&dev, &ds)) return st;
+    FwdArgs a{out, mean, rstd, inp, weight, bias, N, (int)C, 1.0f / float(C), eps,
+              reinterpret_cast<cudaStream_t>(stream), dev, ds->sms};
+    const cudaError_t e = dtype == LN_F32 ? fwd_dispatch<float>(a)
+                                          : fwd_dispatch<lnk::bf16>(a);
+    return status_of(e);
+}
+
+int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
+                const void *inp, const void *weight, const float *mean, const float *rstd,
+                int64_t N, int64_t C, int dtype, ln_stream_t stream) {
+    if (int st = check_shape(N, C)) return st;
+    if (dtype != LN_F32 && dtype != LN_BF16) return LN_ERR_DTYPE;
+    if (!dweight || !dbias) return LN_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(dweight, 0, size_t(C) * sizeof(float), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dbias, 0, size_t(C) * sizeof(float), s);
+        return status_of(e);
+    }
+    if (!dinp || !dout || !inp || !weight || !mean || !rstd) return LN_ERR_NULL;
+    int dev = 0;
+    DeviceState *ds = nullptr;
+    if (int st = current_device(&dev, &ds)) return st;
+    BwdArgs a{dinp, dweight, dbias, dout, inp, weight, mean, rstd, N, (int)C,
+              1.0f / float(C), s, dev, ds->sms, ds->pool};
+    return dtype == LN_F32 ? bwd_dispatch<float>(a) : bwd_dispatch<lnk::bf16>(a);
+}
+
+const char *ln_status_string(int status) {
+    switch (status) {
+        case LN_OK: return "LN_OK: success";
+        case LN_ERR_NULL: return "LN_ERR_NULL: a required pointer is NULL";
+        case LN_ERR_SHAPE: return "LN_ERR_SHAPE: N or C out of range (0 <= N <= 2^40, 1 <= C <= 2^24, N*C <= 2^50)";
+        case LN_ERR_DTYPE: return "LN_ERR_DTYPE: dtype must be LN_F32 (0) or LN_BF16 (1)";
+        case LN_ERR_EPS: return "LN_ERR_EPS: eps must be finite and > 0";
+        case LN_ERR_WORKSPACE: return "LN_ERR_WORKSPACE: backward workspace allocation failed";
+        case LN_ERR_CUDA: return "LN_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+        default: return "unknown ln_status";
+    }
+}
+
+uint64_t ln_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ln_version(void) { return 1; }
+
+}  // extern "C"

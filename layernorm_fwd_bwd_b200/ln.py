@@ -1,0 +1,117 @@
+"""Python binding of libln.so (declared in include/ln.h).
+
+Argument marshalling only: every array argument may be a CUDA ``torch.Tensor``
+(its ``data_ptr()`` is passed), a plain integer device address, or ``None``
+(NULL).  ``stream`` may be a ``torch.cuda.Stream``, a raw ``cudaStream_t``
+integer, or ``None`` for PyTorch's current stream on the current device.
+The caller owns all memory and must make the right device current.
+
+All computation happens in the CUDA library.  If ``libln.so`` has not been
+built, importing this module raises ``ImportError``; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libln.so")
+
+LN_F32 = 0
+LN_BF16 = 1
+
+LN_OK = 0
+LN_ERR_NULL = 1
+LN_ERR_SHAPE = 2
+LN_ERR_DTYPE = 3
+LN_ERR_EPS = 4
+LN_ERR_WORKSPACE = 5
+LN_ERR_CUDA = 6
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with "
+        "`python -m layernorm_fwd_bwd_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_vp, _i64, _int, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+_lib.ln_forward.restype = _int
+_lib.ln_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _int, _vp]
+_lib.ln_backward.restype = _int
+_lib.ln_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _vp]
+_lib.ln_status_string.restype = ctypes.c_char_p
+_lib.ln_status_string.argtypes = [_int]
+_lib.ln_launch_count.restype = ctypes.c_uint64
+_lib.ln_launch_count.argtypes = []
+_lib.ln_version.restype = _int
+_lib.ln_version.argtypes = []
+
+
+class LNError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(ln_status_string(status))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def ln_status_string(status: int) -> str:
+    return _lib.ln_status_string(int(status)).decode()
+
+
+def launch_count() -> int:
+    return int(_lib.ln_launch_count())
+
+
+def version() -> int:
+    return int(_lib.ln_version())
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int) -> None:
+    if rc != LN_OK:
+        raise LNError(rc)
+
+
+def ln_forward(out, mean, rstd, inp, weight, bias, N: int, C: int, eps: float,
+               dtype: int, stream=None) -> None:
+    """out, mean, rstd <- LayerNorm(inp; weight, bias, eps) over N rows of C."""
+    _check(_lib.ln_forward(_ptr(out), _ptr(mean), _ptr(rstd), _ptr(inp),
+                           _ptr(weight), _ptr(bias), int(N), int(C), float(eps),
+                           int(dtype), _stream(stream)))
+
+
+def ln_backward(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
+                C: int, dtype: int, stream=None) -> None:
+    """dinp, dweight, dbias <- analytical LayerNorm backward of dout."""
+    _check(_lib.ln_backward(_ptr(dinp), _ptr(dweight), _ptr(dbias), _ptr(dout),
+                            _ptr(inp), _ptr(weight), _ptr(mean), _ptr(rstd),
+                            int(N), int(C), int(dtype), _stream(stream)))
+
+
+def raw_forward(*args) -> int:
+    """Call ln_forward with already-marshalled arguments; returns the status."""
+    return int(_lib.ln_forward(*args))
+
+
+def raw_backward(*args) -> int:
+    """Call ln_backward with already-marshalled arguments; returns the status."""
+    return int(_lib.ln_backward(*args))

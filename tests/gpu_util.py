@@ -1,0 +1,68 @@
+"""Device-side helpers shared by the GPU tests: move seeded storage arrays to
+the GPU, call the C ABI through the binding, and bring results back as
+float64.  No LayerNorm arithmetic here."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+from layernorm_fwd_bwd_b200 import workloads as wl
+
+DT = {"f32": 0, "bf16": 1}
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def ln():
+    from layernorm_fwd_bwd_b200 import build
+    build.build()
+    from layernorm_fwd_bwd_b200 import ln as binding
+    return binding
+
+
+def to_device(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+    bits = np.ascontiguousarray(a, np.uint16).view(np.int16)
+    return torch.from_numpy(bits).to(device).view(torch.bfloat16)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return wl.bf16_bits_to_f64(t.view(torch.int16).numpy().view(np.uint16))
+    return t.numpy().astype(np.float64)
+
+
+def nan_tensor(shape, tdtype, device="cuda") -> torch.Tensor:
+    return torch.full(shape, float("nan"), dtype=tdtype, device=device)
+
+
+def forward(lib, inp, w, b, N, C, eps, dtype, stream=None):
+    out = nan_tensor((N, C), TORCH_DT[dtype])
+    mean = nan_tensor((N,), torch.float32)
+    rstd = nan_tensor((N,), torch.float32)
+    lib.ln_forward(out, mean, rstd, inp, w, b, N, C, eps, DT[dtype], stream)
+    return out, mean, rstd
+
+
+def backward(lib, dout, inp, w, mean, rstd, N, C, dtype, stream=None):
+    dinp = nan_tensor((N, C), TORCH_DT[dtype])
+    dw = nan_tensor((C,), torch.float32)
+    db = nan_tensor((C,), torch.float32)
+    lib.ln_backward(dinp, dw, db, dout, inp, w, mean, rstd, N, C, DT[dtype], stream)
+    return dinp, dw, db
+
+
+def batch_to_device(batch: wl.Batch):
+    d = batch.workload.dtype
+    return (to_device(batch.inp, d), to_device(batch.weight, d),
+            to_device(batch.bias, d), to_device(batch.dout, d))
+
+
+@functools.lru_cache(maxsize=2)
+def full_batch(name: str) -> wl.Batch:
+    """The named workload at its full size (cached: drawing 50M elements takes
+    seconds)."""
+    return wl.generate(wl.WORKLOADS[name])

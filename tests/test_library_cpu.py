@@ -1,0 +1,105 @@
+"""The C-ABI library on a host without a GPU: it builds, loads, exports every
+symbol include/ln.h declares, and rejects bad arguments before it makes any
+CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ln.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from layernorm_fwd_bwd_b200 import build
+    build.build()
+    from layernorm_fwd_bwd_b200 import ln
+    return ln
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ln_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("ln_forward", "ln_backward", "ln_status_string", "ln_launch_count",
+              "ln_version"):
+        assert n in names
+
+
+def test_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.library_path())
+    for name in declared_functions():
+        assert hasattr(so, name), f"{name} not exported"
+    dyn = subprocess.run(["nm", "-D", "--defined-only", lib.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ln_[a-z_0-9]+)$", dyn, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.ln_status_string(code).startswith(
+            ["LN_OK", "LN_ERR_NULL", "LN_ERR_SHAPE", "LN_ERR_DTYPE", "LN_ERR_EPS",
+             "LN_ERR_WORKSPACE", "LN_ERR_CUDA"][code])
+    assert lib.ln_status_string(99) == "unknown ln_status"
+    assert lib.version() == 1
+
+
+def test_host_validation_without_gpu(lib):
+    # Each of these returns before the library touches the CUDA runtime.
+    f = lib.raw_forward
+    nz = 16  # any non-NULL address: never dereferenced on these paths
+    assert f(nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, None) == lib.LN_ERR_SHAPE
+    assert f(nz, nz, nz, nz, nz, nz, 4, 0, 1e-5, 0, None) == lib.LN_ERR_SHAPE
+    assert f(nz, nz, nz, nz, nz, nz, 4, (1 << 24) + 1, 1e-5, 0, None) == lib.LN_ERR_SHAPE
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 2, None) == lib.LN_ERR_DTYPE
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, 0.0, 0, None) == lib.LN_ERR_EPS
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, float("nan"), 0, None) == lib.LN_ERR_EPS
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, float("inf"), 1, None) == lib.LN_ERR_EPS
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, -1e-5, 1, None) == lib.LN_ERR_EPS
+    assert f(None, nz, nz, nz, nz, nz, 4, 8, 1e-5, 0, None) == lib.LN_ERR_NULL
+    assert f(nz, nz, nz, nz, nz, None, 4, 8, 1e-5, 0, None) == lib.LN_ERR_NULL
+    assert f(None, None, None, None, None, None, 0, 8, 1e-5, 0, None) == lib.LN_OK
+    b = lib.raw_backward
+    assert b(nz, nz, nz, nz, nz, nz, nz, nz, -1, 8, 0, None) == lib.LN_ERR_SHAPE
+    assert b(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 7, None) == lib.LN_ERR_DTYPE
+    assert b(nz, None, nz, nz, nz, nz, nz, nz, 4, 8, 0, None) == lib.LN_ERR_NULL
+    assert b(nz, nz, None, nz, nz, nz, nz, nz, 0, 8, 0, None) == lib.LN_ERR_NULL
+    assert lib.launch_count() == 0
+
+
+def test_binding_raises_lnerror(lib):
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_forward(16, 16, 16, 16, 16, 16, -3, 8, 1e-5, 0, stream=0)
+    assert e.value.status == lib.LN_ERR_SHAPE
+
+
+def test_rejects_oversized_products(lib):
+    nz = 16
+    assert lib.raw_forward(nz, nz, nz, nz, nz, nz, 1 << 40, 1 << 11, 1e-5, 0,
+                           None) == lib.LN_ERR_SHAPE
+    assert lib.raw_backward(nz, nz, nz, nz, nz, nz, nz, nz, 1 << 30, 1 << 21, 1,
+                            None) == lib.LN_ERR_SHAPE
+
+
+def test_tolerance_helpers():
+    import numpy as np
+
+    import tolerances as tol
+    ref = np.array([1.0, -2.0, 0.5])
+    assert tol.max_ulps(ref, ref) == 0.0
+    # one bf16 ulp at 1.0 is 2^-7
+    assert tol.max_ulps(ref + np.array([2.0 ** -7, 0, 0]), ref) == 1.0
+    # near-zero values are judged at 2^-8 * max|ref|
+    assert tol.max_ulps(np.array([2.0 ** -15, 1.0]), np.array([0.0, 1.0])) == 1.0
+    assert tol.rel_max(ref * (1 + 1e-6), ref) <= 1.1e-6
+    assert tol.rel_max(np.array([1e-3 + 1e-8]), np.array([1e-3]), scale=1.0) <= 1.1e-8
+    with pytest.raises(AssertionError):
+        tol.check("x", ref * (1 + 1e-4), ref, "f32", "act_fwd")

@@ -1,0 +1,263 @@
+"""Parity of the CUDA library with the CPU oracle, element by element, on the
+same seeded inputs (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as gu
+import oracle
+import tolerances as tol
+from layernorm_fwd_bwd_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return gu.ln()
+
+
+def _forward_parity(lib, batch, label, scaled=False):
+    """scaled: judge against the magnitude of the summands (shapes outside
+    the five workloads); otherwise each tensor's own max-abs."""
+    w = batch.workload
+    N, C, d = batch.inp.shape[0], w.C, w.dtype
+    inp, wt, bs, dout = gu.batch_to_device(batch)
+    out, mean, rstd = gu.forward(lib, inp, wt, bs, N, C, batch.eps, d)
+    ref_out, ref_mean, ref_rstd = oracle.ln_forward(batch.f64("inp"), batch.f64("weight"),
+                                                    batch.f64("bias"), batch.eps)
+    sc = _scales(batch, ref_mean, ref_rstd) if scaled else {}
+    res = [tol.check(f"{label} out", gu.to_f64(out), ref_out, d, "act_fwd"),
+           tol.check(f"{label} mean", gu.to_f64(mean), ref_mean, d, "stats",
+                     sc.get("mean", 0.0)),
+           tol.check(f"{label} rstd", gu.to_f64(rstd), ref_rstd, d, "stats")]
+    return (inp, wt, bs, dout), (out, mean, rstd), (ref_mean, ref_rstd), res
+
+
+def _scales(batch, mean, rstd):
+    return tol.magnitude_scales(batch.f64("inp"), batch.f64("dout"), batch.f64("weight"),
+                                mean, rstd)
+
+
+def _backward_parity(lib, batch, dev, label, ref_stats, scaled=False):
+    """Backward as a function of its arguments: both sides get the same fp32
+    mean/rstd (the oracle's statistics rounded to fp32)."""
+    w = batch.workload
+    N, C, d = batch.inp.shape[0], w.C, w.dtype
+    inp, wt, _, dout = dev
+    mean32 = ref_stats[0].astype(np.float32)
+    rstd32 = ref_stats[1].astype(np.float32)
+    dinp, dw, db = gu.backward(lib, dout, inp, wt, torch.from_numpy(mean32).cuda(),
+                               torch.from_numpy(rstd32).cuda(), N, C, d)
+    r_dinp, r_dw, r_db = oracle.ln_backward(batch.f64("dout"), batch.f64("inp"),
+                                            batch.f64("weight"), mean32, rstd32)
+    sc = _scales(batch, mean32, rstd32) if scaled else {}
+    return [tol.check(f"{label} dinp", gu.to_f64(dinp), r_dinp, d, "act_bwd",
+                      sc.get("dinp", 0.0)),
+            tol.check(f"{label} dweight", gu.to_f64(dw), r_dw, d, "param_grad",
+                      sc.get("dweight", 0.0)),
+            tol.check(f"{label} dbias", gu.to_f64(db), r_db, d, "param_grad",
+                      sc.get("dbias", 0.0))]
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_full_workload_parity(lib, name):
+    """Every element of every output at the full workload sizes, in the launch
+    configuration the benchmark uses: forward vs the oracle; backward as a
+    function of its arguments (both sides get the oracle's statistics rounded
+    to fp32); and, except for the stress workload, the GPU forward feeding the
+    GPU backward against the oracle in double from end to end.  (In the stress
+    workload the fp32 rounding of a mean near 100 alone moves xhat by up to
+    rstd * ulp(100)/2 ~ 4e-4, so there the backward is judged only as a
+    function of its own arguments.)"""
+    batch = gu.full_batch(name)
+    dev, (out, mean, rstd), ref_stats, res = _forward_parity(lib, batch, name)
+    res += _backward_parity(lib, batch, dev, name, ref_stats)
+    w = batch.workload
+    if w.const_row_period:
+        rows = np.arange(w.N) % w.const_row_period == 0
+        # constant rows: deviations are exactly zero, so out == bias bitwise
+        # and mean == the row's value bitwise
+        out_h = gu.to_f64(out)[rows]
+        assert np.array_equal(out_h, np.broadcast_to(batch.f64("bias"), out_h.shape))
+        assert np.array_equal(gu.to_f64(mean)[rows], batch.f64("inp")[rows, 0])
+    else:
+        inp, wt, _, dout = dev
+        dinp, dw, db = gu.backward(lib, dout, inp, wt, mean, rstd, w.N, w.C, w.dtype)
+        r_dinp, r_dw, r_db = oracle.ln_backward(batch.f64("dout"), batch.f64("inp"),
+                                                batch.f64("weight"), ref_stats[0],
+                                                ref_stats[1])
+        res += [tol.check(f"{name} chained dinp", gu.to_f64(dinp), r_dinp, w.dtype, "act_bwd"),
+                tol.check(f"{name} chained dweight", gu.to_f64(dw), r_dw, w.dtype,
+                          "param_grad"),
+                tol.check(f"{name} chained dbias", gu.to_f64(db), r_db, w.dtype,
+                          "param_grad")]
+    print(res)
+
+
+SWEEP_C = [1, 2, 3, 7, 8, 31, 33, 127, 128, 768, 1023, 1024, 1600, 2048, 2056, 4096,
+           8192, 16384, 20000]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("C", SWEEP_C)
+@pytest.mark.parametrize("N", [1, 3, 257])
+def test_shape_sweep(lib, dtype, C, N):
+    """Ragged tails of the vector paths, every row-ownership variant, and the
+    scalar path (C * size not a multiple of 16 bytes, or C past the vector
+    limits)."""
+    batch = wl.custom(dtype, N, C, seed=1000 + C + N)
+    dev, _, ref_stats, _ = _forward_parity(lib, batch, f"{dtype} {N}x{C}", scaled=True)
+    _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("C", [768, 1600, 5])
+def test_misaligned_pointers(lib, dtype, C):
+    """Arrays that start one element past a 16-byte boundary take the scalar
+    path and give the same results."""
+    N = 37
+    batch = wl.custom(dtype, N, C, seed=77)
+    td = gu.TORCH_DT[dtype]
+
+    def shifted(a):
+        t = gu.to_device(a.reshape(-1), dtype)
+        buf = torch.empty(t.numel() + 1, dtype=td, device="cuda")
+        buf[1:] = t
+        return buf[1:]
+
+    inp, wt, bs, dout = (shifted(batch.inp), shifted(batch.weight), shifted(batch.bias),
+                         shifted(batch.dout))
+    assert inp.data_ptr() % 16 != 0
+    outb = torch.empty(N * C + 1, dtype=td, device="cuda")
+    out = outb[1:]
+    mean = torch.empty(N, device="cuda")
+    rstd = torch.empty(N, device="cuda")
+    lib.ln_forward(out, mean, rstd, inp, wt, bs, N, C, batch.eps, gu.DT[dtype])
+    ro, rm, rr = oracle.ln_forward(batch.f64("inp"), batch.f64("weight"),
+                                   batch.f64("bias"), batch.eps)
+    m32, r32 = rm.astype(np.float32), rr.astype(np.float32)
+    sc = _scales(batch, m32, r32)
+    tol.check("out", gu.to_f64(out).reshape(N, C), ro, dtype, "act_fwd")
+    tol.check("mean", gu.to_f64(mean), rm, dtype, "stats", sc["mean"])
+    dinpb = torch.empty(N * C + 1, dtype=td, device="cuda")
+    dw = torch.empty(C, device="cuda")
+    db = torch.empty(C, device="cuda")
+    lib.ln_backward(dinpb[1:], dw, db, dout, inp, wt, torch.from_numpy(m32).cuda(),
+                    torch.from_numpy(r32).cuda(), N, C, gu.DT[dtype])
+    rd, rw, rb = oracle.ln_backward(batch.f64("dout"), batch.f64("inp"),
+                                    batch.f64("weight"), m32, r32)
+    tol.check("dinp", gu.to_f64(dinpb[1:]).reshape(N, C), rd, dtype, "act_bwd", sc["dinp"])
+    tol.check("dweight", gu.to_f64(dw), rw, dtype, "param_grad", sc["dweight"])
+    tol.check("dbias", gu.to_f64(db), rb, dtype, "param_grad", sc["dbias"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("C", [768, 1600, 7, 20000])
+def test_guard_regions_and_full_coverage(lib, dtype, C):
+    """Outputs sit inside larger buffers whose margins hold a sentinel; after
+    both calls the margins are unchanged and no output element is left at
+    its NaN pre-fill."""
+    N = 130
+    G = 256                       # margin elements on each side (keeps 16-B alignment)
+    batch = wl.custom(dtype, N, C, seed=5)
+    inp, wt, bs, dout = gu.batch_to_device(batch)
+    td = gu.TORCH_DT[dtype]
+
+    def guarded(n, tdt):
+        buf = torch.full((n + 2 * G,), float("nan"), dtype=tdt, device="cuda")
+        buf[:G] = 3.25
+        buf[-G:] = -7.5
+        return buf, buf[G:G + n]
+
+    def intact(buf):
+        return bool((buf[:G] == 3.25).all()) and bool((buf[-G:] == -7.5).all())
+
+    ob, out = guarded(N * C, td)
+    mb, mean = guarded(N, torch.float32)
+    rb_, rstd = guarded(N, torch.float32)
+    lib.ln_forward(out, mean, rstd, inp, wt, bs, N, C, batch.eps, gu.DT[dtype])
+    db_, dinp = guarded(N * C, td)
+    wb, dw = guarded(C, torch.float32)
+    bb, dbias = guarded(C, torch.float32)
+    lib.ln_backward(dinp, dw, dbias, dout, inp, wt, mean, rstd, N, C, gu.DT[dtype])
+    torch.cuda.synchronize()
+    for name, buf, view in (("out", ob, out), ("mean", mb, mean), ("rstd", rb_, rstd),
+                            ("dinp", db_, dinp), ("dweight", wb, dw), ("dbias", bb, dbias)):
+        assert intact(buf), f"{name}: write outside its bounds"
+        assert not bool(torch.isnan(view.float()).any()), f"{name}: element not written"
+
+
+@pytest.mark.parametrize("name", ["gpt2_124m_bf16", "stress_fp32_65536x768"])
+def test_deterministic(lib, name):
+    """Same inputs, different launch histories: bitwise-identical outputs."""
+    w = wl.WORKLOADS[name]
+    batch = wl.generate(w, rows=np.arange(8192))
+    inp, wt, bs, dout = gu.batch_to_device(batch)
+    N = 8192
+    results = []
+    for k in range(3):
+        if k == 1:   # perturb: an unrelated call of another shape in between
+            other = wl.custom(w.dtype, 999, 1600, seed=3)
+            oi, ow, ob, od = gu.batch_to_device(other)
+            gu.forward(lib, oi, ow, ob, 999, 1600, 1e-5, w.dtype)
+        stream = torch.cuda.Stream() if k == 2 else torch.cuda.current_stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            out, mean, rstd = gu.forward(lib, inp, wt, bs, N, w.C, batch.eps, w.dtype)
+            dinp, dw, db = gu.backward(lib, dout, inp, wt, mean, rstd, N, w.C, w.dtype)
+        torch.cuda.synchronize()
+        results.append([t.clone() for t in (out, mean, rstd, dinp, dw, db)])
+    def bits(t):
+        return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+    for r in results[1:]:
+        for a, b in zip(results[0], r):
+            assert torch.equal(bits(a), bits(b))
+
+
+def test_empty_batch(lib):
+    C = 64
+    w = torch.ones(C, device="cuda")
+    dw = torch.full((C,), float("nan"), device="cuda")
+    db = torch.full((C,), float("nan"), device="cuda")
+    before = lib.launch_count()
+    lib.ln_forward(None, None, None, None, w, w, 0, C, 1e-5, 0)
+    lib.ln_backward(None, dw, db, None, None, w, None, None, 0, C, 0)
+    torch.cuda.synchronize()
+    assert lib.launch_count() == before
+    assert bool((dw == 0).all()) and bool((db == 0).all())
+
+
+def test_errors_launch_nothing(lib):
+    x = torch.zeros(4, 8, device="cuda")
+    v = torch.zeros(8, device="cuda")
+    s = torch.zeros(4, device="cuda")
+    before = lib.launch_count()
+    for args, status in (
+            ((None, s, s, x, v, v, 4, 8, 1e-5, 0), lib.LN_ERR_NULL),
+            ((x, s, s, x, v, None, 4, 8, 1e-5, 0), lib.LN_ERR_NULL),
+            ((x, s, s, x, v, v, 4, 8, 1e-5, 5), lib.LN_ERR_DTYPE),
+            ((x, s, s, x, v, v, 4, 8, float("nan"), 0), lib.LN_ERR_EPS),
+            ((x, s, s, x, v, v, -4, 8, 1e-5, 0), lib.LN_ERR_SHAPE)):
+        with pytest.raises(lib.LNError) as e:
+            lib.ln_forward(*args)
+        assert e.value.status == status
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_backward(x, v, v, x, x, v, s, None, 4, 8, 0)
+    assert e.value.status == lib.LN_ERR_NULL
+    assert lib.launch_count() == before
+
+
+def test_launch_counts(lib):
+    """One forward launches one kernel; one backward two (row pass, column
+    finalise)."""
+    batch = wl.custom("bf16", 64, 768, seed=9)
+    inp, wt, bs, dout = gu.batch_to_device(batch)
+    c0 = lib.launch_count()
+    out, mean, rstd = gu.forward(lib, inp, wt, bs, 64, 768, 1e-5, "bf16")
+    c1 = lib.launch_count()
+    gu.backward(lib, dout, inp, wt, mean, rstd, 64, 768, "bf16")
+    c2 = lib.launch_count()
+    assert (c1 - c0, c2 - c1) == (1, 2)
