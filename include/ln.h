@@ -75,7 +75,8 @@ typedef enum {
     LN_ERR_DTYPE = 3,      /* dtype is not LN_F32 or LN_BF16 */
     LN_ERR_EPS = 4,        /* eps is not finite, or not > 0 */
     LN_ERR_WORKSPACE = 5,  /* the backward's workspace could not be allocated */
-    LN_ERR_CUDA = 6        /* a CUDA runtime call or launch failed */
+    LN_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
+    LN_ERR_SCRATCH = 7     /* ln_backward_noalloc: C > LN_NOALLOC_MAX_C */
 } ln_status;
 
 /*
@@ -113,6 +114,36 @@ int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
                 const void *inp, const void *weight, const float *mean,
                 const float *rstd, int64_t N, int64_t C, int dtype,
                 ln_stream_t stream);
+
+/*
+ * ln_backward_noalloc: the same computation and arguments as ln_backward, for
+ * callers that cannot allocate device memory.  (No counterpart on the pages
+ * this library follows: it exists for callers, not for the method.)  Who
+ * needs it: programs that reserve all device memory in one arena at start-up
+ * and forbid allocation afterwards, code running inside another allocator
+ * (where an allocation would re-enter it), and hosts whose memory accounting
+ * must not see a second pool.  ln_backward takes its partial sums from a
+ * stream-ordered pool; this variant keeps them in a static device array of
+ * LN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - The first call on a device (made with that device current) looks up the
+ *     array's device address once; make that call before any stream capture.
+ *   - All calls share the one array.  Each call overwrites what it reads, so
+ *     nothing needs clearing, but calls whose kernels overlap on the GPU
+ *     (other streams, other host threads) race on it: serialise them.
+ *   - C > LN_NOALLOC_MAX_C (one partial row of 2*C fp32 must fit) returns
+ *     LN_ERR_SCRATCH without launching; wide rows run on fewer blocks than
+ *     ln_backward would use, so they may be slower.
+ * Results match ln_backward within the library's stated tolerances (the
+ * column sums may be grouped differently when the array caps the grid).
+ */
+#define LN_NOALLOC_SCRATCH_BYTES ((int64_t)4 << 20)
+#define LN_NOALLOC_MAX_C (LN_NOALLOC_SCRATCH_BYTES / 8)
+int ln_backward_noalloc(void *dinp, float *dweight, float *dbias, const void *dout,
+                        const void *inp, const void *weight, const float *mean,
+                        const float *rstd, int64_t N, int64_t C, int dtype,
+                        ln_stream_t stream);
 
 /* Static description of an ln_status value (never NULL). */
 const char *ln_status_string(int status);

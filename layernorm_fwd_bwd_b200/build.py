@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libln.so")
-SOURCES = [os.path.join(CSRC, "ln_api.cu")]
+SOURCES = [os.path.join(CSRC, "ln_api.cu"), os.path.join(CSRC, "ln_noalloc.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, "ln_kernels.cuh"), os.path.join(INCLUDE, "ln.h")]
 
 NVCC_FLAGS = [

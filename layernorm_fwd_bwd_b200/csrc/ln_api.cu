@@ -342,6 +342,11 @@ int check_shape(int64_t N, int64_t C) {
 
 }  // namespace
 
+// Launches made by ln_noalloc.cu count in ln_launch_count() too.
+void ln_internal_count_launches(uint64_t n) {
+    g_launches.fetch_add(n, std::memory_order_relaxed);
+}
+
 extern "C" {
 
 int ln_forward(void *out, float *mean, float *rstd, const void *inp, const void *weight,
@@ -392,6 +397,7 @@ const char *ln_status_string(int status) {
         case LN_ERR_EPS: return "LN_ERR_EPS: eps must be finite and > 0";
         case LN_ERR_WORKSPACE: return "LN_ERR_WORKSPACE: backward workspace allocation failed";
         case LN_ERR_CUDA: return "LN_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+        case LN_ERR_SCRATCH: return "LN_ERR_SCRATCH: C exceeds the static scratch of ln_backward_noalloc";
         default: return "unknown ln_status";
     }
 }

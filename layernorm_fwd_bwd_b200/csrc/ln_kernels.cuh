@@ -447,7 +447,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
 // warp + 8, ... in increasing order, and warp 0 then adds the 8 results in
 // order 0..7.  The order depends on G only, so the result is deterministic.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+static __global__ void __launch_bounds__(256)
 ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
                  const float *__restrict__ partial, int G, int C) {
     pdl_wait_primary();

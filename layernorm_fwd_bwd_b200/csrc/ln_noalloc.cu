@@ -1,0 +1,196 @@
+// ln_noalloc.cu -- ln_backward_noalloc: the LayerNorm backward for callers
+// that cannot allocate device memory.
+//
+// ln_backward draws its per-block partial sums from a stream-ordered memory
+// pool.  Some callers cannot let a library allocate: programs that reserve
+// all device memory in one arena at start-up and forbid allocation afterwards,
+// code that runs inside another allocator (where calling an allocator would
+// re-enter it), and hosts whose memory accounting must not see a second pool.
+// This entry point computes the same result with its partial sums in a
+// file-scope static device array of LN_NOALLOC_SCRATCH_BYTES, which every GPU
+// that loads the library holds until the process exits.  It calls no
+// cudaMalloc, cudaFree or other allocating routine.
+//
+// Set-up: the first call on a device (with that device current) looks up the
+// array's device address with cudaGetSymbolAddress and caches it; make that
+// first call before any stream capture.  In host code the array's name is only
+// a host-side stand-in, never a device address, so kernels are always given
+// the looked-up pointer.
+//
+// Sharing: every call uses the same array and the array keeps the previous
+// call's contents.  Each block overwrites its whole partial row before the
+// finalise reads it, so nothing needs clearing; but calls whose kernels
+// overlap on the GPU (different streams, or several host threads) race on the
+// array and must be serialised by the caller.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/ln.h"
+#include "ln_kernels.cuh"
+
+// Defined in ln_api.cu: adds to the count ln_launch_count() reports.
+void ln_internal_count_launches(uint64_t n);
+
+static __device__ __align__(256) float ln_noalloc_scratch[LN_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kScratchFloats = LN_NOALLOC_SCRATCH_BYTES / sizeof(float);
+
+struct ScratchDevice {
+    std::once_flag once;
+    float *scratch = nullptr;   // device address of ln_noalloc_scratch
+    int sms = 0;
+    cudaError_t err = cudaSuccess;
+};
+ScratchDevice g_sd[kMaxDevices];
+
+// Runs once per device, with that device current.
+cudaError_t scratch_device(int dev, ScratchDevice **out) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    ScratchDevice &d = g_sd[dev];
+    std::call_once(d.once, [&]() {
+        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.scratch),
+                                             ln_noalloc_scratch);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        d.err = e;
+    });
+    *out = &d;
+    return d.err;
+}
+
+struct Args {
+    void *dinp;
+    float *dweight;
+    float *dbias;
+    const void *dout;
+    const void *inp;
+    const void *weight;
+    const float *mean;
+    const float *rstd;
+    int64_t N;
+    int C;
+    float inv_C;
+    cudaStream_t stream;
+    int sms;
+    float *scratch;
+};
+
+template <typename K, typename... Ts>
+cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
+                   bool pdl, Ts... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess) ln_internal_count_launches(1);
+    return e;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+template <typename T, typename K>
+int run(const Args &a, K kern, int threads, size_t smem, int rows_granule) {
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int occ = 0;
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
+    if (e != cudaSuccess || occ < 1) return LN_ERR_CUDA;
+    // one partial row of 2C floats per block, all within the static array
+    int64_t G = std::min<int64_t>(int64_t(a.sms) * occ, ceil_div(a.N, rows_granule));
+    G = std::min<int64_t>(G, kScratchFloats / (2 * int64_t(a.C)));
+    G = std::max<int64_t>(G, 1);
+    const int64_t rows_per_block = ceil_div(a.N, G);
+    G = ceil_div(a.N, rows_per_block);
+    e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
+               a.scratch, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+               static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+               rows_per_block);
+    if (e == cudaSuccess)
+        e = launch(lnk::ln_colsum_kernel, (int)ceil_div(2 * int64_t(a.C), 32), 256, 0,
+                   a.stream, true, a.dweight, a.dbias,
+                   static_cast<const float *>(a.scratch), (int)G, a.C);
+    return e == cudaSuccess ? LN_OK : LN_ERR_CUDA;
+}
+
+template <typename T, int V, int W, int GROUPS>
+int vec(const Args &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    const int nvec = a.C / E;
+    const size_t smem = size_t(nvec) * 16 + (GROUPS > 1 ? 2 * size_t(a.C) * 4 : 0) +
+                        (W > 1 ? 4 * W * sizeof(float) : 0);
+    return run<T>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>, 32 * W * GROUPS, smem, GROUPS);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename T>
+int dispatch(const Args &a) {
+    constexpr int E = lnk::Vec<T>::E;
+    const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.dinp) &&
+                        aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
+    if (vec_ok) {
+        const int nvec = a.C / E;
+        switch ((nvec + 31) / 32) {
+            case 1: return vec<T, 1, 1, 8>(a);
+            case 2: return vec<T, 2, 1, 8>(a);
+            case 3: return vec<T, 3, 1, 8>(a);
+            case 4: return vec<T, 4, 1, 8>(a);
+            case 5: return vec<T, 5, 1, 8>(a);
+            case 6: return vec<T, 6, 1, 8>(a);
+            case 7: return vec<T, 7, 1, 8>(a);
+            case 8: return vec<T, 8, 1, 8>(a);
+            default: break;
+        }
+        if (nvec <= 2 * 128) return vec<T, 4, 2, 1>(a);
+        if (nvec <= 4 * 128) return vec<T, 4, 4, 1>(a);
+        if (nvec <= 8 * 128) return vec<T, 4, 8, 1>(a);
+        if (nvec <= 16 * 128) return vec<T, 4, 16, 1>(a);
+    }
+    const int threads = (int)std::min<int64_t>(512, ceil_div(a.C, 32) * 32);
+    return run<T>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1);
+}
+
+}  // namespace
+
+extern "C" int ln_backward_noalloc(void *dinp, float *dweight, float *dbias,
+                                   const void *dout, const void *inp, const void *weight,
+                                   const float *mean, const float *rstd, int64_t N,
+                                   int64_t C, int dtype, ln_stream_t stream) {
+    if (N < 0 || N > LN_MAX_N || C < 1 || C > LN_MAX_C || N > LN_MAX_ELEMS / C)
+        return LN_ERR_SHAPE;
+    if (dtype != LN_F32 && dtype != LN_BF16) return LN_ERR_DTYPE;
+    if (C > LN_NOALLOC_MAX_C) return LN_ERR_SCRATCH;
+    if (!dweight || !dbias) return LN_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(dweight, 0, size_t(C) * sizeof(float), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dbias, 0, size_t(C) * sizeof(float), s);
+        return e == cudaSuccess ? LN_OK : LN_ERR_CUDA;
+    }
+    if (!dinp || !dout || !inp || !weight || !mean || !rstd) return LN_ERR_NULL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LN_ERR_CUDA;
+    ScratchDevice *sd = nullptr;
+    if (scratch_device(dev, &sd) != cudaSuccess) return LN_ERR_CUDA;
+    Args a{dinp, dweight, dbias, dout, inp, weight, mean, rstd, N, (int)C,
+           1.0f / float(C), s, sd->sms, sd->scratch};
+    return dtype == LN_F32 ? dispatch<float>(a) : dispatch<lnk::bf16>(a);
+}

@@ -27,6 +27,9 @@ LN_ERR_DTYPE = 3
 LN_ERR_EPS = 4
 LN_ERR_WORKSPACE = 5
 LN_ERR_CUDA = 6
+LN_ERR_SCRATCH = 7
+LN_NOALLOC_SCRATCH_BYTES = 4 << 20
+LN_NOALLOC_MAX_C = LN_NOALLOC_SCRATCH_BYTES // 8
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
@@ -39,6 +42,9 @@ _lib.ln_forward.restype = _int
 _lib.ln_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _int, _vp]
 _lib.ln_backward.restype = _int
 _lib.ln_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _vp]
+_lib.ln_backward_noalloc.restype = _int
+_lib.ln_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                     _int, _vp]
 _lib.ln_status_string.restype = ctypes.c_char_p
 _lib.ln_status_string.argtypes = [_int]
 _lib.ln_launch_count.restype = ctypes.c_uint64
@@ -105,6 +111,18 @@ def ln_backward(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
     _check(_lib.ln_backward(_ptr(dinp), _ptr(dweight), _ptr(dbias), _ptr(dout),
                             _ptr(inp), _ptr(weight), _ptr(mean), _ptr(rstd),
                             int(N), int(C), int(dtype), _stream(stream)))
+
+
+def ln_backward_noalloc(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
+                        C: int, dtype: int, stream=None) -> None:
+    """ln_backward for callers that cannot allocate device memory: its partial
+    sums live in a static device array inside the library (4 MiB per GPU),
+    so C is limited to LN_NOALLOC_MAX_C and calls that overlap on the GPU
+    race on that array; the first call on a device must precede any stream
+    capture."""
+    _check(_lib.ln_backward_noalloc(_ptr(dinp), _ptr(dweight), _ptr(dbias), _ptr(dout),
+                                    _ptr(inp), _ptr(weight), _ptr(mean), _ptr(rstd),
+                                    int(N), int(C), int(dtype), _stream(stream)))
 
 
 def raw_forward(*args) -> int:
