@@ -152,6 +152,15 @@ const char *ln_status_string(int status);
  * all streams).  For accounting in benchmarks and tests. */
 uint64_t ln_launch_count(void);
 
+/* Diagnostics: the bits that kernels of this library set on the current
+ * device when one of their bounded waits ran out (1: a consumer gave up on a
+ * stage's data, 2: the producer gave up on a stage's release, 4: a bulk copy
+ * in flight did not land in time).  0 means healthy; any other value means
+ * the results of the calls since the last clear are not to be trusted.
+ * Writes the bits to *bits and, when clear != 0, resets them.  Synchronises
+ * the current device.  Returns LN_OK, LN_ERR_NULL or LN_ERR_CUDA. */
+int ln_device_status(unsigned int *bits, int clear);
+
 /* Library ABI version: 1. */
 int ln_version(void);
 

@@ -18,7 +18,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libln.so")
 SOURCES = [os.path.join(CSRC, "ln_api.cu"), os.path.join(CSRC, "ln_noalloc.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, "ln_kernels.cuh"), os.path.join(INCLUDE, "ln.h")]
+DEPENDS = SOURCES + [os.path.join(CSRC, "ln_kernels.cuh"), os.path.join(CSRC, "ln_select.cuh"),
+                     os.path.join(CSRC, "ln_tma.cuh"),
+                     os.path.join(CSRC, "ln_tile.cuh"),
+                     os.path.join(INCLUDE, "ln.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -3,15 +3,9 @@
 //
 // Geometry.  Every kernel runs on a persistent grid of (SM count) x (resident
 // blocks per SM, from the occupancy calculator for the exact block size and
-// shared memory), capped by the number of rows.  Row ownership:
-//   C * sizeof(T) a multiple of 16 and all activation/parameter arrays
-//   16-byte aligned  -> vectorised kernels:
-//       C / E <= 32 * Vmax      one warp per row, 8 rows per 256-thread block,
-//                               V = ceil(C / E / 32) vectors per lane;
-//       C / E <= 32 * 32 * 4    W = 2..32 warps per row (2..16 in the backward),
-//                               4 vectors per thread;
-//   otherwise                -> scalar kernels (any alignment, any C).
-// where E = 16 / sizeof(T) elements per vector.
+// shared memory), capped by the number of rows.  Arrays that are all 16-byte
+// aligned, with C * sizeof(T) a multiple of 16, take the vectorised kernels
+// (variant chosen in ln_select.cuh); any other call takes the scalar kernels.
 //
 // Workspace.  The backward needs G * 2C fp32 partial sums (G = its grid).
 // They are drawn stream-ordered from a memory pool that the library creates
@@ -29,23 +23,25 @@
 
 #include "../../include/ln.h"
 #include "ln_kernels.cuh"
+#include "ln_select.cuh"
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kRowsPerBlockW1 = 8;       // row groups per block, one warp per row
-constexpr int kMaxVecPerLaneFwd = 8;
-constexpr int kMaxVecPerLaneBwd = 8;
-constexpr int kMultiWarpVec = 4;         // vectors per thread with W > 1
 constexpr size_t kMaxWorkspaceBytes = size_t(256) << 20;
 
 std::atomic<uint64_t> g_launches{0};
+
+// Bits set by kernels that gave up a bounded wait (see ln_tma.cuh); read with
+// ln_device_status().
+static __device__ unsigned int ln_status_word;
 
 struct DeviceState {
     std::once_flag once;
     int sms = 0;
     int max_smem_optin = 0;
     cudaMemPool_t pool = nullptr;
+    unsigned int *status = nullptr;   // device address of ln_status_word
     cudaError_t init_error = cudaSuccess;
 };
 DeviceState g_dev[kMaxDevices];
@@ -69,6 +65,8 @@ cudaError_t device_state(int dev, DeviceState **out) {
             uint64_t keep = UINT64_MAX;
             e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
         }
+        if (e == cudaSuccess)
+            e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), ln_status_word);
         d.init_error = e;
     });
     *out = &d;
@@ -140,6 +138,63 @@ cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t st
     return e;
 }
 
+// Launch with a 1-D thread-block cluster of `cluster` blocks.
+template <typename K, typename... Args>
+cudaError_t launch_cluster(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
+                           int cluster, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+// Whether a cluster launch of `kernel` can be resident at all (cached).
+template <typename K>
+cudaError_t cluster_fits(K kernel, int dev, int threads, size_t smem, int cluster, bool *fits) {
+    const OccKey key{reinterpret_cast<const void *>(kernel), dev, -cluster, smem + threads};
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        auto it = g_occ.find(key);
+        if (it != g_occ.end()) {
+            *fits = it->second > 0;
+            return cudaSuccess;
+        }
+    }
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    g_occ[key] = n;
+    *fits = n > 0;
+    return cudaSuccess;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -162,24 +217,70 @@ struct FwdArgs {
     cudaStream_t stream;
     int dev;
     int sms;
+    unsigned int *status;
 };
 
-template <typename T, int V, int W, int GROUPS>
-cudaError_t fwd_vec(const FwdArgs &a) {
-    constexpr int E = lnk::Vec<T>::E;
-    auto kern = lnk::ln_fwd_vec_kernel<T, V, W, GROUPS>;
-    const int threads = 32 * W * GROUPS;
-    const int nvec = a.C / E;
-    const size_t smem = size_t(2) * nvec * 16 + (W > 1 ? 2 * W * sizeof(float) : 0);
-    int occ = 0;
-    cudaError_t e = blocks_per_sm(kern, a.dev, threads, smem, &occ);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>(ceil_div(a.N, GROUPS), int64_t(a.sms) * occ);
-    return launch(kern, (int)grid, threads, smem, a.stream, false,
-                  static_cast<T *>(a.out), a.mean, a.rstd, static_cast<const T *>(a.inp),
-                  static_cast<const T *>(a.weight), static_cast<const T *>(a.bias), a.N,
-                  a.C, a.inv_C, a.eps);
-}
+template <typename T>
+struct FwdVec {
+    const FwdArgs &a;
+    cudaError_t err = cudaSuccess;
+    template <int V, int W, int GROUPS>
+    void run() {
+        if constexpr (W == 1 && LN_FWD_STYLE == 2) {
+            if (ceil_div(a.N, lnk::kTileWarps * lnk::kTileFwdTiles) <= INT32_MAX) {
+                run_tile<V>();
+                return;
+            }
+        }
+        if constexpr (W == 1 && LN_FWD_STYLE >= 1) {
+            run_tma<V>();
+            return;
+        }
+        auto kern = lnk::ln_fwd_vec_kernel<T, V, W, GROUPS>;
+        const int threads = 32 * W * GROUPS;
+        const size_t smem = lnk::fwd_vec_smem<W, GROUPS>(a.C);
+        int occ = 0;
+        err = blocks_per_sm(kern, a.dev, threads, smem, &occ);
+        if (err != cudaSuccess) return;
+        const int64_t grid = std::min<int64_t>(ceil_div(a.N, GROUPS), int64_t(a.sms) * occ);
+        err = launch(kern, (int)grid, threads, smem, a.stream, false,
+                     static_cast<T *>(a.out), a.mean, a.rstd,
+                     static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
+                     static_cast<const T *>(a.bias), a.N, a.C, a.inv_C, a.eps);
+    }
+    template <int V>
+    void run_tile() {
+        constexpr int NW = lnk::kTileWarps;
+        constexpr int TL = lnk::kTileFwdTiles;
+        auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL>;
+        const int threads = 32 * NW;
+        const size_t smem = lnk::fwd_tile_smem<T, NW, TL>(a.C);
+        int occ = 0;
+        err = blocks_per_sm(kern, a.dev, threads, smem, &occ);   // also sets the smem limit
+        if (err != cudaSuccess) return;
+        const int64_t grid = ceil_div(a.N, NW * TL);
+        err = launch(kern, (int)grid, threads, smem, a.stream, false,
+                     static_cast<T *>(a.out), a.mean, a.rstd,
+                     static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
+                     static_cast<const T *>(a.bias), a.N, a.C, a.inv_C, a.eps, a.status);
+    }
+    template <int V>
+    void run_tma() {
+        constexpr int NC = lnk::kTmaFwdConsumers;
+        constexpr int S = lnk::FwdStages<V>::value;
+        auto kern = lnk::ln_fwd_tma_kernel<T, V, NC, S>;
+        const int threads = 32 * (NC + 1);
+        const size_t smem = lnk::fwd_tma_smem<T, NC, S>(a.C);
+        int occ = 0;
+        err = blocks_per_sm(kern, a.dev, threads, smem, &occ);
+        if (err != cudaSuccess) return;
+        const int64_t grid = std::min<int64_t>(ceil_div(a.N, NC), int64_t(a.sms) * occ);
+        err = launch(kern, (int)grid, threads, smem, a.stream, false,
+                     static_cast<T *>(a.out), a.mean, a.rstd,
+                     static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
+                     static_cast<const T *>(a.bias), a.N, a.C, a.inv_C, a.eps, a.status);
+    }
+};
 
 template <typename T, bool BLOCK_ROW>
 cudaError_t fwd_scalar(const FwdArgs &a) {
@@ -202,25 +303,8 @@ cudaError_t fwd_dispatch(const FwdArgs &a) {
     const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.out) &&
                         aligned16(a.inp) && aligned16(a.weight) && aligned16(a.bias);
     if (vec_ok) {
-        const int nvec = a.C / E;
-        if (nvec <= 32 * kMaxVecPerLaneFwd) {
-            switch ((nvec + 31) / 32) {
-                case 1: return fwd_vec<T, 1, 1, kRowsPerBlockW1>(a);
-                case 2: return fwd_vec<T, 2, 1, kRowsPerBlockW1>(a);
-                case 3: return fwd_vec<T, 3, 1, kRowsPerBlockW1>(a);
-                case 4: return fwd_vec<T, 4, 1, kRowsPerBlockW1>(a);
-                case 5: return fwd_vec<T, 5, 1, kRowsPerBlockW1>(a);
-                case 6: return fwd_vec<T, 6, 1, kRowsPerBlockW1>(a);
-                case 7: return fwd_vec<T, 7, 1, kRowsPerBlockW1>(a);
-                default: return fwd_vec<T, 8, 1, kRowsPerBlockW1>(a);
-            }
-        }
-        const int per_warp = 32 * kMultiWarpVec;
-        if (nvec <= 2 * per_warp) return fwd_vec<T, kMultiWarpVec, 2, 1>(a);
-        if (nvec <= 4 * per_warp) return fwd_vec<T, kMultiWarpVec, 4, 1>(a);
-        if (nvec <= 8 * per_warp) return fwd_vec<T, kMultiWarpVec, 8, 1>(a);
-        if (nvec <= 16 * per_warp) return fwd_vec<T, kMultiWarpVec, 16, 1>(a);
-        if (nvec <= 32 * per_warp) return fwd_vec<T, kMultiWarpVec, 32, 1>(a);
+        FwdVec<T> v{a};
+        if (lnk::visit_fwd_vec<T>(a.C / E, v)) return v.err;
     }
     if (a.C <= 1024) return fwd_scalar<T, false>(a);
     return fwd_scalar<T, true>(a);
@@ -244,21 +328,26 @@ struct BwdArgs {
     int dev;
     int sms;
     cudaMemPool_t pool;
+    unsigned int *status;
 };
 
-// Runs the row kernel on G blocks of `rows_per_block` consecutive rows, then
-// the fixed-order column finalise (programmatic dependent launch).
-template <typename T, typename K>
-int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule) {
+// Runs the row kernel on G blocks, then the fixed-order column finalise
+// (programmatic dependent launch).  Block b of the row kernel owns
+// `per_block` consecutive units of `unit_rows` rows; TMA kernels also take the
+// device status word.
+template <typename T, bool TMA, typename K>
+int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule,
+            int unit_rows) {
     int occ = 0;
     if (blocks_per_sm(kern, a.dev, threads, smem, &occ) != cudaSuccess) return LN_ERR_CUDA;
+    const int64_t units = ceil_div(a.N, unit_rows);
     int64_t G = std::min<int64_t>(int64_t(a.sms) * occ, ceil_div(a.N, rows_granule));
     // keep the partial sums within kMaxWorkspaceBytes (matters only for very
     // wide rows, where fewer, longer-running blocks are the price)
     G = std::min<int64_t>(G, int64_t(kMaxWorkspaceBytes / (size_t(a.C) * 2 * sizeof(float))));
     G = std::max<int64_t>(G, 1);
-    const int64_t rows_per_block = ceil_div(a.N, G);
-    G = ceil_div(a.N, rows_per_block);
+    const int64_t per_block = ceil_div(units, G);
+    G = ceil_div(units, per_block);
 
     float *partial = nullptr;
     const size_t ws_bytes = size_t(G) * 2 * size_t(a.C) * sizeof(float);
@@ -267,35 +356,100 @@ int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule
         cudaGetLastError();   // clear the non-sticky allocation error
         return LN_ERR_WORKSPACE;
     }
-    cudaError_t e = launch(kern, (int)G, threads, smem, a.stream, false,
-                           static_cast<T *>(a.dinp), partial,
-                           static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
-                           static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C,
-                           a.inv_C, rows_per_block);
+    cudaError_t e;
+    if constexpr (TMA) {
+        e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
+                   partial, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                   static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+                   per_block, a.status);
+    } else {
+        e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
+                   partial, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                   static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+                   per_block * unit_rows);
+    }
     if (e == cudaSuccess) {
         const int cblocks = (int)ceil_div(2 * int64_t(a.C), 32);
-        e = launch(lnk::ln_colsum_kernel, cblocks, 256, 0, a.stream, true, a.dweight,
-                   a.dbias, static_cast<const float *>(partial), (int)G, a.C);
+        e = launch(lnk::ln_colsum_kernel, cblocks, lnk::kColsumThreads, 0, a.stream, true,
+                   a.dweight, a.dbias, static_cast<const float *>(partial), (int)G, a.C);
     }
     const cudaError_t ef = cudaFreeAsync(partial, a.stream);
     if (e == cudaSuccess) e = ef;
     return status_of(e);
 }
 
-template <typename T, int V, int W, int GROUPS>
-int bwd_vec(const BwdArgs &a) {
-    constexpr int E = lnk::Vec<T>::E;
-    const int threads = 32 * W * GROUPS;
-    const int nvec = a.C / E;
-    const size_t smem = size_t(nvec) * 16 + (GROUPS > 1 ? 2 * size_t(a.C) * 4 : 0) +
-                        (W > 1 ? 4 * W * sizeof(float) : 0);
-    return bwd_run<T>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>, threads, smem, GROUPS);
+// One-shot tile backward: clusters of kTileCluster blocks, one partial row per
+// cluster, then the fixed-order finalise.  Returns -1 when the cluster shape
+// cannot be resident (the caller then takes the persistent kernels).
+template <typename T, int V>
+int bwd_tile_run(const BwdArgs &a) {
+    constexpr int NW = lnk::kTileWarps;
+    constexpr int TL = lnk::kTileBwdTiles;
+    constexpr int CL = lnk::kTileCluster;
+    auto kern = lnk::ln_bwd_tile_kernel<T, V, NW, TL, CL>;
+    const int threads = 32 * NW;
+    const size_t smem = lnk::bwd_tile_smem<T, NW, TL>(a.C);
+    const int64_t blocks = ceil_div(ceil_div(a.N, NW * TL), CL) * CL;
+    if (blocks > INT32_MAX) return -1;
+    bool fits = false;
+    if (cluster_fits(kern, a.dev, threads, smem, CL, &fits) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    if (!fits) return -1;
+    const int64_t clusters = blocks / CL;
+    float *partial = nullptr;
+    const size_t ws_bytes = size_t(clusters) * 2 * size_t(a.C) * sizeof(float);
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), ws_bytes, a.pool,
+                                a.stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LN_ERR_WORKSPACE;
+    }
+    cudaError_t e = launch_cluster(kern, (int)blocks, threads, smem, a.stream, CL,
+                                   static_cast<T *>(a.dinp), partial,
+                                   static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                                   static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C,
+                                   a.inv_C, a.status);
+    if (e == cudaSuccess) {
+        const int cblocks = (int)ceil_div(2 * int64_t(a.C), 32);
+        e = launch(lnk::ln_colsum_kernel, cblocks, lnk::kColsumThreads, 0, a.stream, true,
+                   a.dweight, a.dbias, static_cast<const float *>(partial), (int)clusters, a.C);
+    }
+    const cudaError_t ef = cudaFreeAsync(partial, a.stream);
+    if (e == cudaSuccess) e = ef;
+    return status_of(e);
 }
+
+template <typename T>
+struct BwdVec {
+    const BwdArgs &a;
+    int status = LN_OK;
+    template <int V, int W, int GROUPS>
+    void run() {
+        if constexpr (W == 1 && LN_BWD_STYLE == 2) {
+            const int st = bwd_tile_run<T, V>(a);
+            if (st >= 0) {
+                status = st;
+                return;
+            }
+        }
+        if constexpr (W == 1 && LN_BWD_STYLE >= 1) {
+            constexpr int NC = lnk::kTmaBwdConsumers;
+            constexpr int S = lnk::BwdStages<V, NC>::value;
+            status = bwd_run<T, true>(a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0>, 32 * (NC + 1),
+                                      lnk::bwd_tma_smem<T, NC, S>(a.C), NC, NC);
+        } else {
+            status = bwd_run<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
+                                       32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
+                                       GROUPS, 1);
+        }
+    }
+};
 
 template <typename T>
 int bwd_scalar(const BwdArgs &a) {
     int threads = (int)std::min<int64_t>(512, ceil_div(a.C, 32) * 32);
-    return bwd_run<T>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1);
+    return bwd_run<T, false>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1, 1);
 }
 
 template <typename T>
@@ -304,26 +458,8 @@ int bwd_dispatch(const BwdArgs &a) {
     const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.dinp) &&
                         aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
     if (vec_ok) {
-        const int nvec = a.C / E;
-        if (nvec <= 32 * kMaxVecPerLaneBwd) {
-            switch ((nvec + 31) / 32) {
-                case 1: return bwd_vec<T, 1, 1, kRowsPerBlockW1>(a);
-                case 2: return bwd_vec<T, 2, 1, kRowsPerBlockW1>(a);
-                case 3: return bwd_vec<T, 3, 1, kRowsPerBlockW1>(a);
-                case 4: return bwd_vec<T, 4, 1, kRowsPerBlockW1>(a);
-                case 5: return bwd_vec<T, 5, 1, kRowsPerBlockW1>(a);
-                case 6: return bwd_vec<T, 6, 1, kRowsPerBlockW1>(a);
-                case 7: return bwd_vec<T, 7, 1, kRowsPerBlockW1>(a);
-                default: return bwd_vec<T, 8, 1, kRowsPerBlockW1>(a);
-            }
-        }
-        const int per_warp = 32 * kMultiWarpVec;
-        if (nvec <= 2 * per_warp) return bwd_vec<T, kMultiWarpVec, 2, 1>(a);
-        if (nvec <= 4 * per_warp) return bwd_vec<T, kMultiWarpVec, 4, 1>(a);
-        if (nvec <= 8 * per_warp) return bwd_vec<T, kMultiWarpVec, 8, 1>(a);
-        if (nvec <= 16 * per_warp) return bwd_vec<T, kMultiWarpVec, 16, 1>(a);
-        // 1024-thread blocks would cap registers at 64 and spill the column
-        // accumulators: wider rows take the scalar path.
+        BwdVec<T> v{a};
+        if (lnk::visit_bwd_vec<T>(a.C / E, v)) return v.status;
     }
     return bwd_scalar<T>(a);
 }
@@ -347,6 +483,14 @@ void ln_internal_count_launches(uint64_t n) {
     g_launches.fetch_add(n, std::memory_order_relaxed);
 }
 
+// Device address of the status word on the current device (nullptr on error).
+unsigned int *ln_internal_status_word() {
+    int dev = 0;
+    DeviceState *ds = nullptr;
+    if (current_device(&dev, &ds) != LN_OK) return nullptr;
+    return ds->status;
+}
+
 extern "C" {
 
 int ln_forward(void *out, float *mean, float *rstd, const void *inp, const void *weight,
@@ -361,7 +505,7 @@ int ln_forward(void *out, float *mean, float *rstd, const void *inp, const void 
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
     FwdArgs a{out, mean, rstd, inp, weight, bias, N, (int)C, 1.0f / float(C), eps,
-              reinterpret_cast<cudaStream_t>(stream), dev, ds->sms};
+              reinterpret_cast<cudaStream_t>(stream), dev, ds->sms, ds->status};
     const cudaError_t e = dtype == LN_F32 ? fwd_dispatch<float>(a)
                                           : fwd_dispatch<lnk::bf16>(a);
     return status_of(e);
@@ -384,7 +528,7 @@ int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
     BwdArgs a{dinp, dweight, dbias, dout, inp, weight, mean, rstd, N, (int)C,
-              1.0f / float(C), s, dev, ds->sms, ds->pool};
+              1.0f / float(C), s, dev, ds->sms, ds->pool, ds->status};
     return dtype == LN_F32 ? bwd_dispatch<float>(a) : bwd_dispatch<lnk::bf16>(a);
 }
 
@@ -403,6 +547,19 @@ const char *ln_status_string(int status) {
 }
 
 uint64_t ln_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ln_device_status(unsigned int *bits, int clear) {
+    if (!bits) return LN_ERR_NULL;
+    int dev = 0;
+    DeviceState *ds = nullptr;
+    if (int st = current_device(&dev, &ds)) return st;
+    if (cudaMemcpy(bits, ds->status, sizeof(unsigned int), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+        return LN_ERR_CUDA;
+    if (clear && cudaMemset(ds->status, 0, sizeof(unsigned int)) != cudaSuccess)
+        return LN_ERR_CUDA;
+    return LN_OK;
+}
 
 int ln_version(void) { return 1; }
 

@@ -179,12 +179,156 @@ __device__ __forceinline__ void pdl_wait_primary() {
 }
 
 // ---------------------------------------------------------------------------
+// Packed fp32 pairs.  Blackwell executes add/sub/mul/fma on two fp32 values
+// held in one 64-bit register as a single instruction (PTX .f32x2, sm_100+),
+// each lane rounded exactly as the scalar instruction would round it.  The
+// element math below runs on such pairs, which halves its instruction count.
+// ---------------------------------------------------------------------------
+typedef unsigned long long f32x2;   // {lo, hi}
+
+__device__ __forceinline__ f32x2 pair(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void split(f32x2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float hsum(f32x2 v) {
+    float lo, hi;
+    split(v, lo, hi);
+    return lo + hi;
+}
+
+// A 16-byte vector as P = E/2 pairs, and back (bf16 rounded to nearest-even).
+__device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[2]) {
+    p[0] = pair(__uint_as_float(v.x), __uint_as_float(v.y));
+    p[1] = pair(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+__device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[4]) {
+    p[0] = pair(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+    p[1] = pair(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    p[2] = pair(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
+    p[3] = pair(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+}
+__device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[2]) {
+    float a, b, c, d;
+    split(p[0], a, b);
+    split(p[1], c, d);
+    return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c),
+                      __float_as_uint(d));
+}
+__device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[4]) {
+    float f[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) split(p[k], f[2 * k], f[2 * k + 1]);
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+// P pairs of fp32 values from shared memory (16-byte aligned address).
+template <int P>
+__device__ __forceinline__ void smem_pairs(const float *src, f32x2 (&p)[P]) {
+    const ulonglong2 *q = reinterpret_cast<const ulonglong2 *>(src);
+#pragma unroll
+    for (int k = 0; k < P / 2; ++k) {
+        const ulonglong2 u = q[k];
+        p[2 * k] = u.x;
+        p[2 * k + 1] = u.y;
+    }
+}
+
+// Barrier over the TPR threads of one row group (barrier 0 is the block's;
+// groups use 1 .. GROUPS).
+template <int TPR, int GROUPS>
+__device__ __forceinline__ void group_sync(int group) {
+    if constexpr (GROUPS == 1) {
+        __syncthreads();
+    } else {
+        asm volatile("bar.sync %0, %1;" ::"r"(group + 1), "r"(TPR) : "memory");
+    }
+}
+
+// Sum over the W warps of one row group.  `slot` holds 2W floats private to
+// the group; callers alternate slots so that a slot is never rewritten before
+// every thread of the group has read it.
+template <int W, int GROUPS>
+__device__ __forceinline__ float group_sum(float v, float *slot, int group, int warp,
+                                           int lane) {
+    v = warp_sum(v);
+    if constexpr (W == 1) {
+        return v;
+    } else {
+        if (lane == 0) slot[warp] = v;
+        group_sync<32 * W, GROUPS>(group);
+        float tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < W; ++k) tot += slot[k];
+        return tot;
+    }
+}
+
+template <int W, int GROUPS>
+__device__ __forceinline__ void group_sum2(float &a, float &b, float *slot, int group,
+                                           int warp, int lane) {
+    warp_sum2(a, b);
+    if constexpr (W > 1) {
+        if (lane == 0) {
+            slot[warp] = a;
+            slot[W + warp] = b;
+        }
+        group_sync<32 * W, GROUPS>(group);
+        a = 0.f;
+        b = 0.f;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            a += slot[k];
+            b += slot[W + k];
+        }
+    }
+}
+
+// Shared memory of the vectorised kernels (bytes), shared by every launcher.
+template <int W, int GROUPS>
+__host__ __device__ constexpr size_t fwd_vec_smem(int C) {
+    // weight and bias as fp32, then [GROUPS][2 slots][W] reduction floats
+    return size_t(2) * C * 4 + (W > 1 ? size_t(GROUPS) * 2 * W * 4 : 0);
+}
+template <int W, int GROUPS>
+__host__ __device__ constexpr size_t bwd_vec_smem(int C) {
+    // weight as fp32, the combine buffer [GROUPS/2][2C], then
+    // [GROUPS][2 slots][2W] reduction floats
+    return size_t(C) * 4 + (GROUPS > 1 ? size_t(GROUPS / 2) * 2 * C * 4 : 0) +
+           (W > 1 ? size_t(GROUPS) * 4 * W * 4 : 0);
+}
+
+// ---------------------------------------------------------------------------
 // Forward, vectorised path.
 //
-// A row is owned by TPR = 32*W threads; thread t holds 16-byte vectors
-// j = t + i*TPR (i < V) of the row.  W == 1: GROUPS rows per block, one warp
-// per row, shuffle-only reductions.  W > 1: one row per block iteration.
-// Rows are distributed round-robin over a persistent grid.
+// A row is owned by TPR = 32*W threads (a row group); thread t of the group
+// holds 16-byte vectors j = t + i*TPR (i < V) of the row; a block holds
+// GROUPS groups.  Rows go round-robin over a persistent grid.  The row is
+// loaded once, turned into deviations from the pivot x[r, 0] and kept in
+// registers as fp32 pairs through both reductions.
 // Requirements (checked by the host): inp, out, weight, bias 16-byte aligned,
 // C * sizeof(T) a multiple of 16, C / E <= V * TPR.
 // ---------------------------------------------------------------------------
@@ -193,20 +337,16 @@ __global__ void __launch_bounds__(32 * W * GROUPS)
 ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                   const T *__restrict__ inp, const T *__restrict__ weight,
                   const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps) {
-    static_assert(W == 1 || GROUPS == 1, "multi-warp rows run one row per block");
     constexpr int E = Vec<T>::E;
+    constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
     extern __shared__ __align__(16) unsigned char smem[];
     const int nvec = C / E;
-    uint4 *s_w = reinterpret_cast<uint4 *>(smem);
-    uint4 *s_b = s_w + nvec;
-    float *s_red = reinterpret_cast<float *>(s_b + nvec);   // [2][W] when W > 1
-
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(weight);
-    const uint4 *b4 = reinterpret_cast<const uint4 *>(bias);
-    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-        s_w[i] = __ldg(w4 + i);
-        s_b[i] = __ldg(b4 + i);
+    float *s_w = reinterpret_cast<float *>(smem);
+    float *s_b = s_w + C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        s_w[c] = to_f32(weight[c]);
+        s_b[c] = to_f32(bias[c]);
     }
     __syncthreads();
 
@@ -214,6 +354,7 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
     const int t = threadIdx.x - group * TPR;
     const int warp = t >> 5;
     const int lane = threadIdx.x & 31;
+    float *s_red = s_b + C + group * 2 * W;      // [2][W] of this group (W > 1)
 
     for (int64_t r = (int64_t)blockIdx.x * GROUPS + group; r < N;
          r += (int64_t)gridDim.x * GROUPS) {
@@ -226,55 +367,56 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
         }
         float pivot;
         if constexpr (W == 1) {
-            float f[E];
-            unpack(xv[0], f);            // lane 0 holds columns 0 .. E-1
-            pivot = __shfl_sync(0xffffffffu, f[0], 0);
+            float lo, hi;
+            f32x2 p0[P];
+            to_pairs(xv[0], p0);            // lane 0 holds columns 0 .. E-1
+            split(p0[0], lo, hi);
+            pivot = __shfl_sync(0xffffffffu, lo, 0);
         } else {
             pivot = to_f32(inp[r * C]);
         }
+        const f32x2 K = pair(pivot, pivot);
 
-        float s = 0.f;
+        f32x2 d[V][P];
+        f32x2 acc = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            if (t + i * TPR < nvec) {
-                float f[E];
-                unpack(xv[i], f);
+            const bool ok = t + i * TPR < nvec;
+            to_pairs(xv[i], d[i]);
 #pragma unroll
-                for (int e = 0; e < E; ++e) s += f[e] - pivot;
+            for (int k = 0; k < P; ++k) {
+                d[i][k] = sub2(d[i][k], K);
+                if (ok) acc = add2(acc, d[i][k]);
             }
         }
-        s = row_sum<W>(s, s_red, warp, lane);
-        const float mean_d = s * inv_C;         // mean - pivot
+        const float mean_d = group_sum<W, GROUPS>(hsum(acc), s_red, group, warp, lane) * inv_C;
+        const f32x2 M = pair(mean_d, mean_d);
 
-        float q = 0.f;
+        f32x2 q = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            if (t + i * TPR < nvec) {
-                float f[E];
-                unpack(xv[i], f);
+            const bool ok = t + i * TPR < nvec;
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float d = (f[e] - pivot) - mean_d;
-                    q += d * d;
-                }
+            for (int k = 0; k < P; ++k) {
+                d[i][k] = sub2(d[i][k], M);          // x - mean, from the pivot
+                if (ok) q = fma2(d[i][k], d[i][k], q);
             }
         }
-        q = row_sum<W>(q, s_red + W, warp, lane);
-        const float rs = rsqrtf(q * inv_C + eps);
+        const float var = group_sum<W, GROUPS>(hsum(q), s_red + W, group, warp, lane) * inv_C;
+        const float rs = rsqrtf(var + eps);
+        const f32x2 R = pair(rs, rs);
 
         uint4 *yr = reinterpret_cast<uint4 *>(out) + r * nvec;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + i * TPR;
             if (j < nvec) {
-                float f[E], wf[E], bf[E], o[E];
-                unpack(xv[i], f);
-                unpack(s_w[j], wf);
-                unpack(s_b[j], bf);
+                f32x2 wp[P], bp[P], o[P];
+                smem_pairs<P>(s_w + j * E, wp);
+                smem_pairs<P>(s_b + j * E, bp);
 #pragma unroll
-                for (int e = 0; e < E; ++e)
-                    o[e] = ((f[e] - pivot) - mean_d) * rs * wf[e] + bf[e];
-                __stcs(yr + j, pack(o));
+                for (int k = 0; k < P; ++k) o[k] = fma2(mul2(d[i][k], R), wp[k], bp[k]);
+                __stcs(yr + j, from_pairs(o));
             }
         }
         if (t == 0) {
@@ -288,44 +430,47 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
 // Backward, vectorised path.  Same row ownership as the forward.  Block b
 // owns rows [b*rows_per_block, (b+1)*rows_per_block); its row groups take
 // rows row0+g, row0+g+GROUPS, ...  Each thread accumulates dout*xhat and dout
-// for its own columns over all its rows in registers.  At the end the row
-// groups are added in order 0, 1, ..., GROUPS-1 and the block writes
-// partial[b][0:C] (dweight part) and partial[b][C:2C] (dbias part).
+// for its own columns over all its rows, as fp32 pairs in registers.  At the
+// end the groups are added pairwise in a fixed tree (g += g + GROUPS/2, then
+// g += g + GROUPS/4, ...) and group 0 writes partial[b][0:C] (dweight part)
+// and partial[b][C:2C] (dbias part).
+//   dinp = rstd * (g - mean(g) - xhat * mean(g xhat)) is evaluated as
+//   fma(g, rstd, fma(xhat, -rstd*mean(g xhat), -rstd*mean(g))).
 // ---------------------------------------------------------------------------
 template <typename T, int V, int W, int GROUPS>
-__global__ void __launch_bounds__(32 * W * GROUPS)
+__global__ void __launch_bounds__(32 * W * GROUPS, 32 * W * GROUPS <= 256 ? 2 : 1)
 ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ dout, const T *__restrict__ inp,
                   const T *__restrict__ weight, const float *__restrict__ mean,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                   int64_t rows_per_block) {
-    static_assert(W == 1 || GROUPS == 1, "multi-warp rows run one row per block");
     constexpr int E = Vec<T>::E;
+    constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
     extern __shared__ __align__(16) unsigned char smem[];
     const int nvec = C / E;
-    uint4 *s_w = reinterpret_cast<uint4 *>(smem);
-    float *s_acc = reinterpret_cast<float *>(s_w + nvec);            // [2C] if GROUPS > 1
-    float *s_red = s_acc + (GROUPS > 1 ? 2 * C : 0);                 // [2][2W] if W > 1
+    float *s_w = reinterpret_cast<float *>(smem);
+    float *s_acc = s_w + C;                                   // [GROUPS/2][2C]
+    float *s_red0 = s_acc + (GROUPS > 1 ? (GROUPS / 2) * 2 * C : 0);
 
     pdl_launch_dependents();
 
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(weight);
-    for (int i = threadIdx.x; i < nvec; i += blockDim.x) s_w[i] = __ldg(w4 + i);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) s_w[c] = to_f32(weight[c]);
     __syncthreads();
 
     const int group = threadIdx.x / TPR;
     const int t = threadIdx.x - group * TPR;
     const int warp = t >> 5;
     const int lane = threadIdx.x & 31;
+    float *s_red = s_red0 + group * 4 * W;                    // [2][2W] of this group
 
-    float acc_w[V][E], acc_b[V][E];
+    f32x2 acc_w[V][P], acc_b[V][P];
 #pragma unroll
     for (int i = 0; i < V; ++i)
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            acc_w[i][e] = 0.f;
-            acc_b[i][e] = 0.f;
+        for (int k = 0; k < P; ++k) {
+            acc_w[i][k] = pair(0.f, 0.f);
+            acc_b[i][k] = pair(0.f, 0.f);
         }
 
     const int64_t row0 = (int64_t)blockIdx.x * rows_per_block;
@@ -348,124 +493,156 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
         }
         const float m = __ldg(mean + r);
         const float s = __ldg(rstd + r);
+        const f32x2 M = pair(m, m);
+        const f32x2 S = pair(s, s);
 
-        float s1 = 0.f, s2 = 0.f;
+        f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + i * TPR;
             if (j < nvec) {
-                float x[E], dy[E], wf[E];
-                unpack(xv[i], x);
-                unpack(dv[i], dy);
-                unpack(s_w[j], wf);
+                f32x2 x[P], dy[P], wp[P];
+                to_pairs(xv[i], x);
+                to_pairs(dv[i], dy);
+                smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float xh = (x[e] - m) * s;
-                    const float g = dy[e] * wf[e];
-                    s1 += g;
-                    s2 += g * xh;
+                for (int k = 0; k < P; ++k) {
+                    const f32x2 xh = mul2(sub2(x[k], M), S);
+                    const f32x2 g = mul2(dy[k], wp[k]);
+                    s1 = add2(s1, g);
+                    s2 = fma2(g, xh, s2);
                 }
             }
         }
-        row_sum2<W>(s1, s2, s_red + parity * 2 * W, warp, lane);
+        float a = hsum(s1), b = hsum(s2);
+        group_sum2<W, GROUPS>(a, b, s_red + parity * 2 * W, group, warp, lane);
         parity ^= 1;
-        const float a = s1 * inv_C;     // mean of g
-        const float c = s2 * inv_C;     // mean of g * xhat
+        const float na = -s * (a * inv_C);      // -rstd * mean(g)
+        const float nc = -s * (b * inv_C);      // -rstd * mean(g xhat)
+        const f32x2 NA = pair(na, na);
+        const f32x2 NC = pair(nc, nc);
 
         uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + i * TPR;
             if (j < nvec) {
-                float x[E], dy[E], wf[E], o[E];
-                unpack(xv[i], x);
-                unpack(dv[i], dy);
-                unpack(s_w[j], wf);
+                f32x2 x[P], dy[P], wp[P], o[P];
+                to_pairs(xv[i], x);
+                to_pairs(dv[i], dy);
+                smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float xh = (x[e] - m) * s;
-                    const float g = dy[e] * wf[e];
-                    o[e] = s * (g - a - xh * c);
-                    acc_w[i][e] += dy[e] * xh;
-                    acc_b[i][e] += dy[e];
+                for (int k = 0; k < P; ++k) {
+                    const f32x2 xh = mul2(sub2(x[k], M), S);
+                    const f32x2 g = mul2(dy[k], wp[k]);
+                    o[k] = fma2(g, S, fma2(xh, NC, NA));
+                    acc_w[i][k] = fma2(dy[k], xh, acc_w[i][k]);
+                    acc_b[i][k] = add2(acc_b[i][k], dy[k]);
                 }
-                __stcs(gr + j, pack(o));
+                __stcs(gr + j, from_pairs(o));
             }
         }
     }
 
-    float *pblk = partial + (int64_t)blockIdx.x * 2 * C;
-    if constexpr (GROUPS == 1) {
+    // Fixed-order tree over the row groups: at each level, groups
+    // [h, 2h) park their sums in s_acc and groups [0, h) add them.
+    if constexpr (GROUPS > 1) {
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int j = t + i * TPR;
-            if (j < nvec) {
-                float4 *pw = reinterpret_cast<float4 *>(pblk + j * E);
-                float4 *pb = reinterpret_cast<float4 *>(pblk + C + j * E);
-#pragma unroll
-                for (int k = 0; k < E / 4; ++k) {
-                    pw[k] = make_float4(acc_w[i][4 * k], acc_w[i][4 * k + 1],
-                                        acc_w[i][4 * k + 2], acc_w[i][4 * k + 3]);
-                    pb[k] = make_float4(acc_b[i][4 * k], acc_b[i][4 * k + 1],
-                                        acc_b[i][4 * k + 2], acc_b[i][4 * k + 3]);
-                }
-            }
-        }
-    } else {
-        for (int gi = 0; gi < GROUPS; ++gi) {
-            if (group == gi) {
+        for (int h = GROUPS / 2; h >= 1; h /= 2) {
+            if (group >= h && group < 2 * h) {
+                float *dst = s_acc + (group - h) * 2 * C;
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     const int j = t + i * TPR;
                     if (j < nvec) {
+                        ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(dst + j * E);
+                        ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(dst + C + j * E);
 #pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            const int col = j * E + e;
-                            if (gi == 0) {
-                                s_acc[col] = acc_w[i][e];
-                                s_acc[C + col] = acc_b[i][e];
-                            } else {
-                                s_acc[col] += acc_w[i][e];
-                                s_acc[C + col] += acc_b[i][e];
-                            }
+                        for (int k = 0; k < P / 2; ++k) {
+                            pw[k] = make_ulonglong2(acc_w[i][2 * k], acc_w[i][2 * k + 1]);
+                            pb[k] = make_ulonglong2(acc_b[i][2 * k], acc_b[i][2 * k + 1]);
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            if (group < h) {
+                const float *src = s_acc + group * 2 * C;
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int j = t + i * TPR;
+                    if (j < nvec) {
+                        f32x2 pw[P], pb[P];
+                        smem_pairs<P>(src + j * E, pw);
+                        smem_pairs<P>(src + C + j * E, pb);
+#pragma unroll
+                        for (int k = 0; k < P; ++k) {
+                            acc_w[i][k] = add2(acc_w[i][k], pw[k]);
+                            acc_b[i][k] = add2(acc_b[i][k], pb[k]);
                         }
                     }
                 }
             }
             __syncthreads();
         }
-        const float4 *src = reinterpret_cast<const float4 *>(s_acc);
-        float4 *dst = reinterpret_cast<float4 *>(pblk);
-        for (int k = threadIdx.x; k < (2 * C) / 4; k += blockDim.x) dst[k] = src[k];
+    }
+    if (group == 0) {
+        float *pblk = partial + (int64_t)blockIdx.x * 2 * C;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int j = t + i * TPR;
+            if (j < nvec) {
+                ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(pblk + j * E);
+                ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(pblk + C + j * E);
+#pragma unroll
+                for (int k = 0; k < P / 2; ++k) {
+                    pw[k] = make_ulonglong2(acc_w[i][2 * k], acc_w[i][2 * k + 1]);
+                    pb[k] = make_ulonglong2(acc_b[i][2 * k], acc_b[i][2 * k + 1]);
+                }
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Column finalise: dweight[c] = sum_b partial[b][c], dbias[c] =
-// sum_b partial[b][C + c], b = 0 .. G-1.  A block covers 32 of the 2C
-// flattened columns; its 8 warps each sum the partial rows b = warp,
-// warp + 8, ... in increasing order, and warp 0 then adds the 8 results in
-// order 0..7.  The order depends on G only, so the result is deterministic.
+// sum_b partial[b][C + c], b = 0 .. G-1.  A block of kColsumThreads covers 32
+// of the 2C flattened columns with S = kColsumThreads/32 slices: slice y sums
+// the partial rows b = y, y + S, ... in increasing order (16 loads issued
+// before their adds), then slice 0 adds the S slice sums in order.  The order
+// depends on G only, so the result is deterministic.
 // ---------------------------------------------------------------------------
-static __global__ void __launch_bounds__(256)
+constexpr int kColsumThreads = 1024;
+
+static __global__ void __launch_bounds__(kColsumThreads)
 ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
                  const float *__restrict__ partial, int G, int C) {
+    constexpr int S = kColsumThreads / 32;
     pdl_wait_primary();
-    __shared__ float s[8][33];
+    __shared__ float s[S][33];
     const int tx = threadIdx.x & 31;
     const int ty = threadIdx.x >> 5;
     const int64_t twoC = 2 * (int64_t)C;
     const int64_t j = (int64_t)blockIdx.x * 32 + tx;
     float acc = 0.f;
     if (j < twoC) {
-        for (int b = ty; b < G; b += 8) acc += partial[(int64_t)b * twoC + j];
+        for (int b0 = ty; b0 < G; b0 += S * 16) {
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int b = b0 + S * q;
+                v[q] = b < G ? partial[(int64_t)b * twoC + j] : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) acc += v[q];
+        }
     }
     s[ty][tx] = acc;
     __syncthreads();
     if (ty == 0 && j < twoC) {
         float tot = s[0][tx];
 #pragma unroll
-        for (int k = 1; k < 8; ++k) tot += s[k][tx];
+        for (int k = 1; k < S; ++k) tot += s[k][tx];
         if (j < C)
             dweight[j] = tot;
         else

@@ -31,9 +31,12 @@
 
 #include "../../include/ln.h"
 #include "ln_kernels.cuh"
+#include "ln_select.cuh"
 
-// Defined in ln_api.cu: adds to the count ln_launch_count() reports.
+// Defined in ln_api.cu: adds to the count ln_launch_count() reports, and the
+// device status word of the current device.
 void ln_internal_count_launches(uint64_t n);
+unsigned int *ln_internal_status_word();
 
 static __device__ __align__(256) float ln_noalloc_scratch[LN_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 
@@ -80,6 +83,7 @@ struct Args {
     cudaStream_t stream;
     int sms;
     float *scratch;
+    unsigned int *status;
 };
 
 template <typename K, typename... Ts>
@@ -104,8 +108,11 @@ cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t st
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-template <typename T, typename K>
-int run(const Args &a, K kern, int threads, size_t smem, int rows_granule) {
+// Row kernel on G blocks (block b owns `per_block` consecutive units of
+// `unit_rows` rows), then the fixed-order column finalise.
+template <typename T, bool TMA, typename K>
+int run_kernel(const Args &a, K kern, int threads, size_t smem, int rows_granule,
+               int unit_rows) {
     cudaError_t e = cudaSuccess;
     if (smem > 48 * 1024)
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -114,30 +121,102 @@ int run(const Args &a, K kern, int threads, size_t smem, int rows_granule) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
     if (e != cudaSuccess || occ < 1) return LN_ERR_CUDA;
     // one partial row of 2C floats per block, all within the static array
+    const int64_t units = ceil_div(a.N, unit_rows);
     int64_t G = std::min<int64_t>(int64_t(a.sms) * occ, ceil_div(a.N, rows_granule));
     G = std::min<int64_t>(G, kScratchFloats / (2 * int64_t(a.C)));
     G = std::max<int64_t>(G, 1);
-    const int64_t rows_per_block = ceil_div(a.N, G);
-    G = ceil_div(a.N, rows_per_block);
-    e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
-               a.scratch, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
-               static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
-               rows_per_block);
+    const int64_t per_block = ceil_div(units, G);
+    G = ceil_div(units, per_block);
+    if constexpr (TMA) {
+        e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
+                   a.scratch, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                   static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+                   per_block, a.status);
+    } else {
+        e = launch(kern, (int)G, threads, smem, a.stream, false, static_cast<T *>(a.dinp),
+                   a.scratch, static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                   static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+                   per_block * unit_rows);
+    }
     if (e == cudaSuccess)
-        e = launch(lnk::ln_colsum_kernel, (int)ceil_div(2 * int64_t(a.C), 32), 256, 0,
-                   a.stream, true, a.dweight, a.dbias,
+        e = launch(lnk::ln_colsum_kernel, (int)ceil_div(2 * int64_t(a.C), 32),
+                   lnk::kColsumThreads, 0, a.stream, true, a.dweight, a.dbias,
                    static_cast<const float *>(a.scratch), (int)G, a.C);
     return e == cudaSuccess ? LN_OK : LN_ERR_CUDA;
 }
 
-template <typename T, int V, int W, int GROUPS>
-int vec(const Args &a) {
-    constexpr int E = lnk::Vec<T>::E;
-    const int nvec = a.C / E;
-    const size_t smem = size_t(nvec) * 16 + (GROUPS > 1 ? 2 * size_t(a.C) * 4 : 0) +
-                        (W > 1 ? 4 * W * sizeof(float) : 0);
-    return run<T>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>, 32 * W * GROUPS, smem, GROUPS);
+// One-shot tile backward with cluster partials in the static array; -1 when
+// the partial rows do not fit there or the cluster shape cannot be resident.
+template <typename T, int V>
+int run_tile(const Args &a) {
+    constexpr int NW = lnk::kTileWarps;
+    constexpr int TL = lnk::kTileBwdTiles;
+    constexpr int CL = lnk::kTileCluster;
+    auto kern = lnk::ln_bwd_tile_kernel<T, V, NW, TL, CL>;
+    const int threads = 32 * NW;
+    const size_t smem = lnk::bwd_tile_smem<T, NW, TL>(a.C);
+    const int64_t blocks = ceil_div(ceil_div(a.N, NW * TL), CL) * CL;
+    const int64_t clusters = blocks / CL;
+    if (blocks > INT32_MAX || clusters * 2 * int64_t(a.C) > kScratchFloats) return -1;
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+    if (e != cudaSuccess || nclusters < 1) {
+        cudaGetLastError();
+        return -1;
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(a.dinp), a.scratch,
+                           static_cast<const T *>(a.dout), static_cast<const T *>(a.inp),
+                           static_cast<const T *>(a.weight), a.mean, a.rstd, a.N, a.C, a.inv_C,
+                           a.status);
+    if (e == cudaSuccess) {
+        ln_internal_count_launches(1);
+        e = launch(lnk::ln_colsum_kernel, (int)ceil_div(2 * int64_t(a.C), 32),
+                   lnk::kColsumThreads, 0, a.stream, true, a.dweight, a.dbias,
+                   static_cast<const float *>(a.scratch), (int)clusters, a.C);
+    }
+    return e == cudaSuccess ? LN_OK : LN_ERR_CUDA;
 }
+
+template <typename T>
+struct Vec {
+    const Args &a;
+    int status = LN_OK;
+    template <int V, int W, int GROUPS>
+    void run() {
+        if constexpr (W == 1 && LN_BWD_STYLE == 2) {
+            const int st = run_tile<T, V>(a);
+            if (st >= 0) {
+                status = st;
+                return;
+            }
+        }
+        if constexpr (W == 1 && LN_BWD_STYLE >= 1) {
+            constexpr int NC = lnk::kTmaBwdConsumers;
+            constexpr int S = lnk::BwdStages<V, NC>::value;
+            status = run_kernel<T, true>(a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0>, 32 * (NC + 1),
+                                         lnk::bwd_tma_smem<T, NC, S>(a.C), NC, NC);
+        } else {
+            status = run_kernel<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
+                                          32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
+                                          GROUPS, 1);
+        }
+    }
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -147,25 +226,11 @@ int dispatch(const Args &a) {
     const bool vec_ok = (int64_t(a.C) * sizeof(T)) % 16 == 0 && aligned16(a.dinp) &&
                         aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
     if (vec_ok) {
-        const int nvec = a.C / E;
-        switch ((nvec + 31) / 32) {
-            case 1: return vec<T, 1, 1, 8>(a);
-            case 2: return vec<T, 2, 1, 8>(a);
-            case 3: return vec<T, 3, 1, 8>(a);
-            case 4: return vec<T, 4, 1, 8>(a);
-            case 5: return vec<T, 5, 1, 8>(a);
-            case 6: return vec<T, 6, 1, 8>(a);
-            case 7: return vec<T, 7, 1, 8>(a);
-            case 8: return vec<T, 8, 1, 8>(a);
-            default: break;
-        }
-        if (nvec <= 2 * 128) return vec<T, 4, 2, 1>(a);
-        if (nvec <= 4 * 128) return vec<T, 4, 4, 1>(a);
-        if (nvec <= 8 * 128) return vec<T, 4, 8, 1>(a);
-        if (nvec <= 16 * 128) return vec<T, 4, 16, 1>(a);
+        Vec<T> v{a};
+        if (lnk::visit_bwd_vec<T>(a.C / E, v)) return v.status;
     }
     const int threads = (int)std::min<int64_t>(512, ceil_div(a.C, 32) * 32);
-    return run<T>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1);
+    return run_kernel<T, false>(a, lnk::ln_bwd_scalar_kernel<T>, threads, 0, 1, 1);
 }
 
 }  // namespace
@@ -190,7 +255,9 @@ extern "C" int ln_backward_noalloc(void *dinp, float *dweight, float *dbias,
     if (cudaGetDevice(&dev) != cudaSuccess) return LN_ERR_CUDA;
     ScratchDevice *sd = nullptr;
     if (scratch_device(dev, &sd) != cudaSuccess) return LN_ERR_CUDA;
+    unsigned int *status = ln_internal_status_word();
+    if (!status) return LN_ERR_CUDA;
     Args a{dinp, dweight, dbias, dout, inp, weight, mean, rstd, N, (int)C,
-           1.0f / float(C), s, sd->sms, sd->scratch};
+           1.0f / float(C), s, sd->sms, sd->scratch, status};
     return dtype == LN_F32 ? dispatch<float>(a) : dispatch<lnk::bf16>(a);
 }

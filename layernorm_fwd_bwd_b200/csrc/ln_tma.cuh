@@ -1,0 +1,515 @@
+// ln_tma.cuh -- LayerNorm forward and backward fed by a TMA bulk-copy ring.
+//
+// Why: the register-resident kernels keep at most one row per warp in flight
+// (1.5 KB for a bf16 row of 768), and a warp spends most of each row on
+// arithmetic, so a bf16 launch cannot keep enough bytes in flight to reach
+// the HBM roofline.  Here one producer warp per block streams whole tiles of
+// consecutive rows (one contiguous range of global memory) into a ring of S
+// shared-memory stages with 1-D bulk copies (cp.async.bulk, no multicast),
+// so the bytes in flight live in shared memory (S * tile bytes per block)
+// instead of registers.  Consumer warps take one row each from the stage,
+// compute exactly as the register-resident kernels do, and release the stage.
+//
+// Synchronisation: per stage one "full" mbarrier (producer's expect_tx + the
+// copy's completion) and one "empty" mbarrier (one arrival per consumer warp,
+// after a fence.proxy.async that orders the warp's shared-memory reads before
+// the next bulk copy into the stage).
+// Every wait is bounded (kWaitLimitNs of %globaltimer, and an iteration cap):
+// on expiry the thread records an error bit in *status, stops, and the
+// producer waits (again bounded) for its copies in flight before the block
+// exits.  Nothing here waits on another block.
+#pragma once
+
+#include "ln_kernels.cuh"
+
+namespace lnk {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+constexpr uint32_t kMaxWaitIters = 1u << 30;
+
+// status bits
+constexpr unsigned kStatusWaitFull = 1u;    // a consumer gave up on a stage's data
+constexpr unsigned kStatusWaitEmpty = 2u;   // the producer gave up on a stage's release
+constexpr unsigned kStatusDrain = 4u;       // a copy in flight did not land in time
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Order this thread's generic-proxy shared-memory reads before later
+// async-proxy writes (the next bulk copy into the same stage).  Without it a
+// stage can be refilled before the reads that preceded its release were
+// performed -- a write-after-read race that measurably corrupts rows.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait until the phase of `bar` with the given parity has completed; false
+// if that did not happen within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1; it < kMaxWaitIters; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return false;
+}
+// 1-D bulk copy global -> this block's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Shared memory layout (bytes):
+//   [0, 128)            full[S], empty[S] mbarriers (S <= 8)
+//   [128, 128 + A)      fp32 parameters: weight (+ bias in the forward), A = n*C*4 rounded up
+//   [.., + S * stage)   the ring; stage = rows * row_bytes * (1 fwd, 2 bwd)
+template <typename T>
+__host__ __device__ constexpr size_t tma_ring_offset(int C, int nparams) {
+    return 128 + align128(size_t(nparams) * C * 4);
+}
+template <typename T, int NC, int S>
+__host__ __device__ constexpr size_t fwd_tma_smem(int C) {
+    return tma_ring_offset<T>(C, 2) + size_t(S) * NC * C * sizeof(T);
+}
+template <typename T, int NC, int S>
+__host__ __device__ constexpr size_t bwd_tma_smem(int C) {
+    // weight as fp32 (read twice per row: unpacking bf16 there costs more
+    // issue slots than the wider shared-memory reads); the ring is reused for
+    // the end-of-block combine: at most NC/2 parked warps (rounded up) of 2C
+    // floats each
+    const size_t ring = size_t(S) * NC * 2 * C * sizeof(T);
+    const size_t comb = size_t((NC + 1) / 2) * 2 * C * 4;
+    return tma_ring_offset<T>(C, 1) + (ring > comb ? ring : comb);
+}
+
+// Producer side, shared by both kernels: stream tiles k = 0, 1, ... of this
+// block (tile index tile_of(k)) into the ring.  Before returning -- after the
+// last tile, or after recording an error -- it waits (bounded) until its
+// last copies have landed, so the block never exits with a copy still
+// writing into its shared memory.
+template <int S, typename TileOf, typename Issue>
+__device__ __forceinline__ void tma_produce(uint64_t *full, uint64_t *empty,
+                                            int64_t ntiles_here, unsigned *status,
+                                            TileOf tile_of, Issue issue) {
+    int64_t k = 0;
+    for (; k < ntiles_here; ++k) {
+        const int st = int(k % S);
+        const int64_t use = k / S;
+        if (use > 0 && !mbar_wait(&empty[st], uint32_t((use - 1) & 1))) {
+            atomicOr(status, kStatusWaitEmpty);
+            break;
+        }
+        issue(tile_of(k), st, &full[st]);
+    }
+    for (int64_t q = (k > S ? k - S : 0); q < k; ++q)
+        if (!mbar_wait(&full[q % S], uint32_t((q / S) & 1))) atomicOr(status, kStatusDrain);
+}
+
+// ---------------------------------------------------------------------------
+// Forward.  Tile = NC consecutive rows (NC consumer warps, one row each);
+// tiles go round-robin over a persistent grid.  Warp NC is the producer.
+// Requirements (checked by the host): inp/out/weight/bias 16-byte aligned,
+// C * sizeof(T) a multiple of 16, C / E <= 32 * V.
+// ---------------------------------------------------------------------------
+template <typename T, int V, int NC, int S>
+__global__ void __launch_bounds__(32 * (NC + 1))
+ln_fwd_tma_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
+                  const T *__restrict__ inp, const T *__restrict__ weight,
+                  const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps,
+                  unsigned *__restrict__ status) {
+    static_assert(S >= 2 && S <= 8, "ring depth");
+    constexpr int E = Vec<T>::E;
+    constexpr int P = E / 2;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + S;
+    float *s_w = reinterpret_cast<float *>(smem + 128);
+    float *s_b = s_w + C;
+    unsigned char *ring = smem + tma_ring_offset<T>(C, 2);
+    const int nvec = C / E;
+    const uint32_t row_bytes = uint32_t(C) * sizeof(T);
+    const uint32_t stage_bytes = NC * row_bytes;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NC);
+        }
+        fence_mbar_init();
+    }
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        s_w[c] = to_f32(weight[c]);
+        s_b[c] = to_f32(bias[c]);
+    }
+    __syncthreads();
+
+    const int64_t ntiles = (N + NC - 1) / NC;
+    const int64_t ntiles_here =
+        blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (warp == NC) {
+        if (lane == 0) {
+            tma_produce<S>(
+                full, empty, ntiles_here, status,
+                [&](int64_t k) { return int64_t(blockIdx.x) + k * gridDim.x; },
+                [&](int64_t tile, int st, uint64_t *bar) {
+                    const int64_t row0 = tile * NC;
+                    const uint32_t bytes = uint32_t(min64(NC, N - row0)) * row_bytes;
+                    mbar_arrive_expect_tx(bar, bytes);
+                    bulk_load(ring + size_t(st) * stage_bytes,
+                              reinterpret_cast<const unsigned char *>(inp) + row0 * row_bytes,
+                              bytes, bar);
+                });
+        }
+        return;
+    }
+
+    for (int64_t k = 0; k < ntiles_here; ++k) {
+        const int st = int(k % S);
+        if (!mbar_wait(&full[st], uint32_t((k / S) & 1))) {
+            if (lane == 0) atomicOr(status, kStatusWaitFull);
+            break;
+        }
+        const int64_t r = (int64_t(blockIdx.x) + k * gridDim.x) * NC + warp;
+        const bool valid = r < N;                   // warp-uniform
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(ring + size_t(st) * stage_bytes + warp * row_bytes);
+        uint4 xv[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int j = lane + 32 * i;
+            xv[i] = (valid && j < nvec) ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();                   // reads done before the refill
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);     // stage slot read: release it
+        if (!valid) continue;
+
+        float pivot;
+        {
+            float lo, hi;
+            f32x2 p0[P];
+            to_pairs(xv[0], p0);
+            split(p0[0], lo, hi);
+            pivot = __shfl_sync(0xffffffffu, lo, 0);
+        }
+        const f32x2 K = pair(pivot, pivot);
+        f32x2 d[V][P];
+        f32x2 acc = pair(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const bool ok = lane + 32 * i < nvec;
+            to_pairs(xv[i], d[i]);
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+                d[i][q] = sub2(d[i][q], K);
+                if (ok) acc = add2(acc, d[i][q]);
+            }
+        }
+        const float mean_d = warp_sum(hsum(acc)) * inv_C;
+        const f32x2 M = pair(mean_d, mean_d);
+        f32x2 sq = pair(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const bool ok = lane + 32 * i < nvec;
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+                d[i][q] = sub2(d[i][q], M);
+                if (ok) sq = fma2(d[i][q], d[i][q], sq);
+            }
+        }
+        const float rs = rsqrtf(warp_sum(hsum(sq)) * inv_C + eps);
+        const f32x2 R = pair(rs, rs);
+        uint4 *yr = reinterpret_cast<uint4 *>(out) + r * nvec;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int j = lane + 32 * i;
+            if (j < nvec) {
+                f32x2 wp[P], bp[P], o[P];
+                smem_pairs<P>(s_w + j * E, wp);
+                smem_pairs<P>(s_b + j * E, bp);
+#pragma unroll
+                for (int q = 0; q < P; ++q) o[q] = fma2(mul2(d[i][q], R), wp[q], bp[q]);
+                __stcs(yr + j, from_pairs(o));
+            }
+        }
+        if (lane == 0) {
+            mean[r] = pivot + mean_d;
+            rstd[r] = rs;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Backward.  Tile = NC consecutive rows (NC = 15 by default: with the
+// producer warp a 512-thread block, one per SM, 128 registers per thread);
+// block b owns tiles
+// [b*tiles_per_block, (b+1)*tiles_per_block).  A stage holds the tile's inp
+// rows followed by its dout rows.  Consumer warp w takes row w of each tile,
+// keeps dout*xhat and dout for its own columns in registers, and at the end
+// the NC warps are added in a fixed tree (as in the register-resident
+// kernel) and warp 0 writes the block's partial row.  mean/rstd of the next
+// row are prefetched one tile ahead.
+// ---------------------------------------------------------------------------
+template <typename T, int V, int NC, int S, bool RR>
+__global__ void __launch_bounds__(32 * (NC + 1), (NC + 1) * 32 <= 256 ? 2 : 1)
+ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
+                  const T *__restrict__ dout, const T *__restrict__ inp,
+                  const T *__restrict__ weight, const float *__restrict__ mean,
+                  const float *__restrict__ rstd, int64_t N, int C, float inv_C,
+                  int64_t tiles_per_block, unsigned *__restrict__ status) {
+    static_assert(S >= 2 && S <= 8, "ring depth");
+    static_assert(NC >= 2 && NC <= 16, "consumer warps");
+    constexpr int E = Vec<T>::E;
+    constexpr int P = E / 2;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + S;
+    float *s_w = reinterpret_cast<float *>(smem + 128);      // weight as fp32
+    unsigned char *ring = smem + tma_ring_offset<T>(C, 1);
+    const int nvec = C / E;
+    const uint32_t row_bytes = uint32_t(C) * sizeof(T);
+    const uint32_t half_bytes = NC * row_bytes;          // inp part of a stage
+    const uint32_t stage_bytes = 2 * half_bytes;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    pdl_launch_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NC);
+        }
+        fence_mbar_init();
+    }
+    for (int c = threadIdx.x; c < C; c += blockDim.x) s_w[c] = to_f32(weight[c]);
+    __syncthreads();
+
+    // Tiles of this block: RR (round-robin) takes tiles b, b + G, b + 2G, ...
+    // so that the blocks in flight cover one compact window of memory;
+    // otherwise a contiguous range of tiles_per_block tiles.  Either is a
+    // fixed assignment, so the column sums stay deterministic.
+    const int64_t ntiles = (N + NC - 1) / NC;
+    const int64_t tile0 = RR ? int64_t(blockIdx.x) : int64_t(blockIdx.x) * tiles_per_block;
+    const int64_t tstep = RR ? int64_t(gridDim.x) : 1;
+    const int64_t ntiles_here =
+        RR ? (tile0 < ntiles ? (ntiles - 1 - tile0) / tstep + 1 : 0)
+           : (tile0 < ntiles ? min64(tiles_per_block, ntiles - tile0) : 0);
+
+    f32x2 acc_w[V][P], acc_b[V][P];
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+            acc_w[i][q] = pair(0.f, 0.f);
+            acc_b[i][q] = pair(0.f, 0.f);
+        }
+
+    if (warp == NC) {
+        if (lane == 0) {
+            tma_produce<S>(
+                full, empty, ntiles_here, status, [&](int64_t k) { return tile0 + k * tstep; },
+                [&](int64_t tile, int st, uint64_t *bar) {
+                    const int64_t row0 = tile * NC;
+                    const uint32_t bytes = uint32_t(min64(NC, N - row0)) * row_bytes;
+                    mbar_arrive_expect_tx(bar, 2 * bytes);
+                    unsigned char *dst = ring + size_t(st) * stage_bytes;
+                    bulk_load(dst, reinterpret_cast<const unsigned char *>(inp) + row0 * row_bytes,
+                              bytes, bar);
+                    bulk_load(dst + half_bytes,
+                              reinterpret_cast<const unsigned char *>(dout) + row0 * row_bytes,
+                              bytes, bar);
+                });
+        }
+    } else {
+        const int64_t rstep = tstep * NC;
+        int64_t r = tile0 * NC + warp;
+        float m_next = 0.f, s_next = 0.f;
+        if (ntiles_here > 0 && r < N) {
+            m_next = __ldg(mean + r);
+            s_next = __ldg(rstd + r);
+        }
+        for (int64_t k = 0; k < ntiles_here; ++k, r += rstep) {
+            const int st = int(k % S);
+            if (!mbar_wait(&full[st], uint32_t((k / S) & 1))) {
+                if (lane == 0) atomicOr(status, kStatusWaitFull);
+                break;
+            }
+            const bool valid = r < N;                 // warp-uniform
+            const float m = m_next, s = s_next;
+            if (k + 1 < ntiles_here && r + rstep < N) {   // next row's statistics
+                m_next = __ldg(mean + r + rstep);
+                s_next = __ldg(rstd + r + rstep);
+            }
+            const unsigned char *stage = ring + size_t(st) * stage_bytes + warp * row_bytes;
+            const uint4 *xs = reinterpret_cast<const uint4 *>(stage);
+            const uint4 *ds = reinterpret_cast<const uint4 *>(stage + half_bytes);
+            uint4 xv[V], dv[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = lane + 32 * i;
+                const bool ok = valid && j < nvec;
+                xv[i] = ok ? xs[j] : make_uint4(0u, 0u, 0u, 0u);
+                dv[i] = ok ? ds[j] : make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();                 // reads done before the refill
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+            if (!valid) continue;
+
+            const f32x2 M = pair(m, m);
+            const f32x2 Sx = pair(s, s);
+            f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = lane + 32 * i;
+                if (j < nvec) {
+                    f32x2 x[P], dy[P], wp[P];
+                    to_pairs(xv[i], x);
+                    to_pairs(dv[i], dy);
+                    smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        const f32x2 xh = mul2(sub2(x[q], M), Sx);
+                        const f32x2 g = mul2(dy[q], wp[q]);
+                        s1 = add2(s1, g);
+                        s2 = fma2(g, xh, s2);
+                    }
+                }
+            }
+            float a = hsum(s1), b = hsum(s2);
+            warp_sum2(a, b);
+            const float na = -s * (a * inv_C);
+            const float nc = -s * (b * inv_C);
+            const f32x2 NA = pair(na, na);
+            const f32x2 NCc = pair(nc, nc);
+            uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = lane + 32 * i;
+                if (j < nvec) {
+                    f32x2 x[P], dy[P], wp[P], o[P];
+                    to_pairs(xv[i], x);
+                    to_pairs(dv[i], dy);
+                    smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        const f32x2 xh = mul2(sub2(x[q], M), Sx);
+                        const f32x2 g = mul2(dy[q], wp[q]);
+                        o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
+                        acc_w[i][q] = fma2(dy[q], xh, acc_w[i][q]);
+                        acc_b[i][q] = add2(acc_b[i][q], dy[q]);
+                    }
+                    __stcs(gr + j, from_pairs(o));
+                }
+            }
+        }
+    }
+
+    // Fixed-order tree over the NC consumer warps: at each level with width h
+    // (the largest power of two below the active count n, then halving),
+    // warps [h, n) park their sums and warps [0, n - h) add them.  The ring
+    // is free again once every warp has passed the first barrier (all copies
+    // were consumed, or drained by the producer).
+    __syncthreads();
+    float *s_acc = reinterpret_cast<float *>(ring);
+    constexpr int kTop = (NC > 8) ? 8 : (NC > 4) ? 4 : (NC > 2) ? 2 : 1;
+    int n = NC;
+#pragma unroll
+    for (int h = kTop; h >= 1; h /= 2) {
+        if (warp >= h && warp < n) {
+            float *dst = s_acc + (warp - h) * 2 * C;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = lane + 32 * i;
+                if (j < nvec) {
+                    ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(dst + j * E);
+                    ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(dst + C + j * E);
+#pragma unroll
+                    for (int q = 0; q < P / 2; ++q) {
+                        pw[q] = make_ulonglong2(acc_w[i][2 * q], acc_w[i][2 * q + 1]);
+                        pb[q] = make_ulonglong2(acc_b[i][2 * q], acc_b[i][2 * q + 1]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (warp < n - h) {
+            const float *src = s_acc + warp * 2 * C;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = lane + 32 * i;
+                if (j < nvec) {
+                    f32x2 pw[P], pb[P];
+                    smem_pairs<P>(src + j * E, pw);
+                    smem_pairs<P>(src + C + j * E, pb);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        acc_w[i][q] = add2(acc_w[i][q], pw[q]);
+                        acc_b[i][q] = add2(acc_b[i][q], pb[q]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        n = h;
+    }
+    if (warp == 0) {
+        float *pblk = partial + (int64_t)blockIdx.x * 2 * C;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int j = lane + 32 * i;
+            if (j < nvec) {
+                ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(pblk + j * E);
+                ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(pblk + C + j * E);
+#pragma unroll
+                for (int q = 0; q < P / 2; ++q) {
+                    pw[q] = make_ulonglong2(acc_w[i][2 * q], acc_w[i][2 * q + 1]);
+                    pb[q] = make_ulonglong2(acc_b[i][2 * q], acc_b[i][2 * q + 1]);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace lnk

@@ -51,6 +51,8 @@ _lib.ln_launch_count.restype = ctypes.c_uint64
 _lib.ln_launch_count.argtypes = []
 _lib.ln_version.restype = _int
 _lib.ln_version.argtypes = []
+_lib.ln_device_status.restype = _int
+_lib.ln_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
 
 
 class LNError(RuntimeError):
@@ -73,6 +75,14 @@ def launch_count() -> int:
 
 def version() -> int:
     return int(_lib.ln_version())
+
+
+def device_status(clear: bool = False) -> int:
+    """Bits set on the current device by kernels whose bounded waits ran out
+    (0: healthy).  Synchronises the device."""
+    bits = ctypes.c_uint(0)
+    _check(_lib.ln_device_status(ctypes.byref(bits), int(bool(clear))))
+    return int(bits.value)
 
 
 def _ptr(x):
