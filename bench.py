@@ -166,6 +166,26 @@ class ClockSampler:
                 "samples": len(inside)}
 
 
+# ------------------------------------------------------------- multi-rank
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    """The largest value of x over all ranks (x itself without a process
+    group).  Used for every timing: the job is as slow as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, bytes_per_rank_step: int, step_seconds: float) -> float:
+    """Whole-job GB/s: every rank moves bytes_per_rank_step per step (weak
+    scaling), and a step takes the slowest rank's time."""
+    return world * bytes_per_rank_step / step_seconds / 1e9
+
+
 # --------------------------------------------------------------------- ours
 
 def run_ours(args, world: int, rank: int, local: int):
@@ -269,10 +289,7 @@ def run_ours(args, world: int, rank: int, local: int):
     total_ms = start.elapsed_time(end)
     fwd_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in events.values())
     bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in events.values())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else run_e2e(args, torch, ln, stream, dev, h_inp, h_dout,
@@ -286,7 +303,7 @@ def run_ours(args, world: int, rank: int, local: int):
 
     fb, bb = w.fwd_bytes(), w.bwd_bytes()
     step_s = total_ms / 1e3 / K
-    value = world * (fb + bb) / step_s / 1e9
+    value = job_throughput(world, fb + bb, step_s)
     peak, peak_kind = hbm_peak()
     bwd_gbs = bb / (bwd_ms / 1e3) / 1e9
     fwd_gbs = fb / (fwd_ms / 1e3) / 1e9
@@ -368,18 +385,13 @@ def run_e2e(args, torch, ln, stream, dev, h_inp, h_dout, h_w, h_b, N, C, tdt, dc
         one()
     end.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev)
     from layernorm_fwd_bwd_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = sum(v.numel() * v.element_size() for v in hout.values())
     step_s = ms / 1e3 / steps
-    return {"value": round(world * (w.fwd_bytes() + w.bwd_bytes()) / step_s / 1e9, 2),
+    return {"value": round(job_throughput(world, w.fwd_bytes() + w.bwd_bytes(), step_s), 2),
             "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps, "ms_per_step": round(ms / steps, 4)}
 
@@ -431,8 +443,9 @@ def run_reference(args, world: int, rank: int):
     from layernorm_fwd_bwd_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
     # calibrate: rows per second of the oracle on a small sample
-    _, per, _ = _oracle_rate(w, 512, 0.0)
-    rows_per_s = 512 / per
+    cal = min(512, w.N)
+    _, per, _ = _oracle_rate(w, cal, 0.0)
+    rows_per_s = cal / per
     budget = 150.0
     rows = int(max(1, min(w.N, rows_per_s * budget / max(1, args.steps + args.warmup))))
     import numpy as np
