@@ -231,6 +231,19 @@ __device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[4]) {
     p[2] = pair(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
     p[3] = pair(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
 }
+// Pair q of a 16-byte vector (q < E/2), unpacked on its own.
+template <typename T>
+__device__ __forceinline__ f32x2 pair_at(const uint4 &v, int q);
+template <>
+__device__ __forceinline__ f32x2 pair_at<float>(const uint4 &v, int q) {
+    return q == 0 ? pair(__uint_as_float(v.x), __uint_as_float(v.y))
+                  : pair(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+template <>
+__device__ __forceinline__ f32x2 pair_at<bf16>(const uint4 &v, int q) {
+    const uint32_t w = q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
+    return pair(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
 __device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[2]) {
     float a, b, c, d;
     split(p[0], a, b);

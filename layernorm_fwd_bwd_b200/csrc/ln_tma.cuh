@@ -397,50 +397,118 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             if (lane == 0) mbar_arrive(&empty[st]);
             if (!valid) continue;
 
-            const f32x2 M = pair(m, m);
-            const f32x2 Sx = pair(s, s);
-            f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
+            // Pass 1 / pass 2.  Where the register budget allows (KEEP_D), pass 1
+            // keeps d = x - mean as fp32 pairs and pass 2 evaluates
+            //   dinp = g*rstd + NA + d*NC,  NA = -rstd*mean(g),
+            //   NC = -rstd^3*mean(g*d)   (xhat = d*rstd),
+            // so pass 2 never unpacks x again; otherwise both passes rebuild
+            // xhat from the packed row.
+            constexpr bool KEEP_D = sizeof(T) == 4 || V <= 3;
+            uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
+            if constexpr (KEEP_D) {
+                // Pass 1: d = x - mean, g = dout * w, S1 = sum g,
+                // S2' = sum g * d (= sum g * xhat / rstd).  d stays in registers as
+                // fp32 pairs for pass 2 when that fits in the register budget
+                // (KEEP_D); otherwise pass 2 recomputes it from the packed row.
+                const f32x2 M = pair(m, m);
+                const f32x2 Sx = pair(s, s);
+                f32x2 d[V][P];
+                f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int j = lane + 32 * i;
-                if (j < nvec) {
-                    f32x2 x[P], dy[P], wp[P];
-                    to_pairs(xv[i], x);
-                    to_pairs(dv[i], dy);
-                    smem_pairs<P>(s_w + j * E, wp);
+                for (int i = 0; i < V; ++i) {
+                    const int j = lane + 32 * i;
+                    f32x2 dq[P];
+                    to_pairs(xv[i], dq);
 #pragma unroll
                     for (int q = 0; q < P; ++q) {
-                        const f32x2 xh = mul2(sub2(x[q], M), Sx);
-                        const f32x2 g = mul2(dy[q], wp[q]);
-                        s1 = add2(s1, g);
-                        s2 = fma2(g, xh, s2);
+                        dq[q] = sub2(dq[q], M);
+                        d[i][q] = dq[q];
+                    }
+                    if (j < nvec) {
+                        f32x2 dy[P], wp[P];
+                        to_pairs(dv[i], dy);
+                        smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                        for (int q = 0; q < P; ++q) {
+                            const f32x2 g = mul2(dy[q], wp[q]);
+                            s1 = add2(s1, g);
+                            s2 = fma2(g, dq[q], s2);
+                        }
                     }
                 }
-            }
-            float a = hsum(s1), b = hsum(s2);
-            warp_sum2(a, b);
-            const float na = -s * (a * inv_C);
-            const float nc = -s * (b * inv_C);
-            const f32x2 NA = pair(na, na);
-            const f32x2 NCc = pair(nc, nc);
-            uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
+                float a = hsum(s1), b = hsum(s2);
+                warp_sum2(a, b);
+                // dinp = rstd*(g - mean(g) - xhat*mean(g*xhat))
+                //      = g*rstd + NA + d*NC,  NA = -rstd*mean(g),
+                //        NC = -rstd^3 * mean(g*d)   (xhat = d*rstd)
+                const float na = -s * (a * inv_C);
+                const float nc = -(s * s) * (s * (b * inv_C));
+                const f32x2 NA = pair(na, na);
+                const f32x2 NCc = pair(nc, nc);
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int j = lane + 32 * i;
-                if (j < nvec) {
-                    f32x2 x[P], dy[P], wp[P], o[P];
-                    to_pairs(xv[i], x);
-                    to_pairs(dv[i], dy);
-                    smem_pairs<P>(s_w + j * E, wp);
+                for (int i = 0; i < V; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < nvec) {
+                        f32x2 wp[P], o[P];
+                        smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
-                    for (int q = 0; q < P; ++q) {
-                        const f32x2 xh = mul2(sub2(x[q], M), Sx);
-                        const f32x2 g = mul2(dy[q], wp[q]);
-                        o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
-                        acc_w[i][q] = fma2(dy[q], xh, acc_w[i][q]);
-                        acc_b[i][q] = add2(acc_b[i][q], dy[q]);
+                        for (int q = 0; q < P; ++q) {
+                            const f32x2 dd = d[i][q];
+                            const f32x2 dy = pair_at<T>(dv[i], q);
+                            const f32x2 g = mul2(dy, wp[q]);
+                            o[q] = fma2(g, Sx, fma2(dd, NCc, NA));
+                            const f32x2 xh = mul2(dd, Sx);
+                            acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
+                            acc_b[i][q] = add2(acc_b[i][q], dy);
+                        }
+                        __stcs(gr + j, from_pairs(o));
                     }
-                    __stcs(gr + j, from_pairs(o));
+                }
+            } else {
+                const f32x2 M = pair(m, m);
+                const f32x2 Sx = pair(s, s);
+                f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < nvec) {
+                        f32x2 x[P], dy[P], wp[P];
+                        to_pairs(xv[i], x);
+                        to_pairs(dv[i], dy);
+                        smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                        for (int q = 0; q < P; ++q) {
+                            const f32x2 xh = mul2(sub2(x[q], M), Sx);
+                            const f32x2 g = mul2(dy[q], wp[q]);
+                            s1 = add2(s1, g);
+                            s2 = fma2(g, xh, s2);
+                        }
+                    }
+                }
+                float a = hsum(s1), b = hsum(s2);
+                warp_sum2(a, b);
+                const float na = -s * (a * inv_C);
+                const float nc = -s * (b * inv_C);
+                const f32x2 NA = pair(na, na);
+                const f32x2 NCc = pair(nc, nc);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < nvec) {
+                        f32x2 x[P], dy[P], wp[P], o[P];
+                        to_pairs(xv[i], x);
+                        to_pairs(dv[i], dy);
+                        smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                        for (int q = 0; q < P; ++q) {
+                            const f32x2 xh = mul2(sub2(x[q], M), Sx);
+                            const f32x2 g = mul2(dy[q], wp[q]);
+                            o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
+                            acc_w[i][q] = fma2(dy[q], xh, acc_w[i][q]);
+                            acc_b[i][q] = add2(acc_b[i][q], dy[q]);
+                        }
+                        __stcs(gr + j, from_pairs(o));
+                    }
                 }
             }
         }
