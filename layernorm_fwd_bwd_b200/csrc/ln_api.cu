@@ -228,7 +228,10 @@ struct FwdVec {
     void run() {
         if constexpr (W == 1 && LN_FWD_STYLE == 2) {
             if (ceil_div(a.N, lnk::kTileWarps * lnk::kTileFwdTiles) <= INT32_MAX) {
-                run_tile<V>();
+                if constexpr (V >= LN_TILE_FWD_W2_FROM_V)
+                    run_tile<(V + 1) / 2, 2>();
+                else
+                    run_tile<V, 1>();
                 return;
             }
         }
@@ -248,17 +251,17 @@ struct FwdVec {
                      static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
                      static_cast<const T *>(a.bias), a.N, a.C, a.inv_C, a.eps);
     }
-    template <int V>
+    template <int V, int RW>
     void run_tile() {
-        constexpr int NW = lnk::kTileWarps;
+        constexpr int NW = lnk::kTileWarps * RW;          // 8 rows per tile either way
         constexpr int TL = lnk::kTileFwdTiles;
-        auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL>;
+        auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL, RW>;
         const int threads = 32 * NW;
-        const size_t smem = lnk::fwd_tile_smem<T, NW, TL>(a.C);
+        const size_t smem = lnk::fwd_tile_smem<T, NW, TL, RW>(a.C);
         int occ = 0;
         err = blocks_per_sm(kern, a.dev, threads, smem, &occ);   // also sets the smem limit
         if (err != cudaSuccess) return;
-        const int64_t grid = ceil_div(a.N, NW * TL);
+        const int64_t grid = ceil_div(a.N, (NW / RW) * TL);
         err = launch(kern, (int)grid, threads, smem, a.stream, false,
                      static_cast<T *>(a.out), a.mean, a.rstd,
                      static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
@@ -433,11 +436,13 @@ struct BwdVec {
                 return;
             }
         }
-        if constexpr (W == 1 && LN_BWD_STYLE >= 1) {
-            constexpr int NC = lnk::kTmaBwdConsumers;
+        if constexpr ((W == 1 || W == 2) && LN_BWD_STYLE >= 1) {
+            constexpr int NC = lnk::BwdRingConsumers<W>::value;
             constexpr int S = lnk::BwdStages<V, NC>::value;
-            status = bwd_run<T, true>(a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0>, 32 * (NC + 1),
-                                      lnk::bwd_tma_smem<T, NC, S>(a.C), NC, NC);
+            constexpr int RT = NC / W;                    // rows per tile
+            status = bwd_run<T, true>(
+                a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
+                lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
         } else {
             status = bwd_run<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
                                        32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),

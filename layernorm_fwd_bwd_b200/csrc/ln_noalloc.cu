@@ -205,11 +205,13 @@ struct Vec {
                 return;
             }
         }
-        if constexpr (W == 1 && LN_BWD_STYLE >= 1) {
-            constexpr int NC = lnk::kTmaBwdConsumers;
+        if constexpr ((W == 1 || W == 2) && LN_BWD_STYLE >= 1) {
+            constexpr int NC = lnk::BwdRingConsumers<W>::value;
             constexpr int S = lnk::BwdStages<V, NC>::value;
-            status = run_kernel<T, true>(a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0>, 32 * (NC + 1),
-                                         lnk::bwd_tma_smem<T, NC, S>(a.C), NC, NC);
+            constexpr int RT = NC / W;                    // rows per tile
+            status = run_kernel<T, true>(
+                a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
+                lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
         } else {
             status = run_kernel<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
                                           32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),

@@ -58,6 +58,16 @@ namespace lnk {
 #endif
 constexpr int kTmaFwdConsumers = LN_TMA_FWD_CONSUMERS;
 constexpr int kTmaBwdConsumers = LN_TMA_BWD_CONSUMERS;
+// consumer warps of the backward ring when W warps share a row
+template <int W> struct BwdRingConsumers {
+    static constexpr int value = (kTmaBwdConsumers / W) * W;
+};
+// forward tile kernel: rows of up to 4 vectors per lane take one warp, wider
+// one-warp rows (5..8 vectors) are split over two warps (fewer registers,
+// more warps per SM)
+#ifndef LN_TILE_FWD_W2_FROM_V
+#define LN_TILE_FWD_W2_FROM_V 5
+#endif
 constexpr int kTileWarps = 8;                 // warps (= rows per tile) per tile block
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
 constexpr int kTileBwdTiles = LN_TILE_BWD_TILES;

@@ -34,9 +34,13 @@ namespace lnk {
 
 // Shared memory: [128 B barriers][params: n * C * sizeof(T), 128-aligned]
 //                [tiles: TILES * NW * row_bytes * arrays][backward: 2C fp32]
-template <typename T, int NW, int TILES>
+template <typename T, int NW, int TILES, int W = 1>
 __host__ __device__ constexpr size_t fwd_tile_smem(int C) {
-    return 128 + align128(size_t(2) * C * sizeof(T)) + size_t(TILES) * NW * C * sizeof(T);
+    // barriers, raw weight + bias, TILES tiles of NW / W rows, and the
+    // row-group exchange slots when rows are shared by W > 1 warps
+    return 128 + align128(size_t(2) * C * sizeof(T)) +
+           align128(size_t(TILES) * (NW / W) * C * sizeof(T)) +
+           (W > 1 ? size_t(NW / W) * 2 * 3 * W * 4 : 0);
 }
 template <typename T, int NW, int TILES>
 __host__ __device__ constexpr size_t bwd_tile_tiles_bytes(int C) {
@@ -58,42 +62,55 @@ __device__ __forceinline__ bool tile_wait(uint64_t *bar, unsigned *status, unsig
 }
 
 // ---------------------------------------------------------------------------
-// Forward.  Requirements (checked by the host): inp/out/weight/bias 16-byte
-// aligned, C * sizeof(T) a multiple of 16, C / E <= 32 * V.
+// Forward.  NW warps; W warps share a row, so a tile holds RT = NW / W rows
+// and the block covers TILES tiles.  Warp w serves row w / W of each tile and
+// vectors j = (w % W) * 32 + lane + i * 32 * W of it.  The pivot is the row's
+// first element, read from shared memory by every warp of the row; with
+// W > 1 the row sums meet through group_exchange (ln_tma.cuh).
+// Requirements (checked by the host): inp/out/weight/bias 16-byte aligned,
+// C * sizeof(T) a multiple of 16, C / E <= 32 * W * V.
 // ---------------------------------------------------------------------------
-template <typename T, int V, int NW, int TILES>
+template <typename T, int V, int NW, int TILES, int W = 1>
 __global__ void __launch_bounds__(32 * NW)
 ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                    const T *__restrict__ inp, const T *__restrict__ weight,
                    const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps,
                    unsigned *__restrict__ status) {
     static_assert(TILES + 1 <= 16, "barriers fit in 128 bytes");
+    static_assert(NW % W == 0 && NW / W <= 15, "row groups");
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
+    constexpr int RT = NW / W;                                // rows per tile
+    constexpr int TPR = 32 * W;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);      // [0]: params, [1+t]: tile t
     const uint32_t row_bytes = uint32_t(C) * sizeof(T);
     unsigned char *s_par = smem + 128;                         // weight then bias, raw
     unsigned char *s_tiles = s_par + align128(size_t(2) * row_bytes);
+    float *s_red = reinterpret_cast<float *>(
+        s_tiles + align128(size_t(TILES) * RT * row_bytes));   // [RT][2][3W] (W > 1)
     const int nvec = C / E;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row0 = int64_t(blockIdx.x) * (NW * TILES);
+    const int group = warp / W;
+    const int sub = warp - group * W;
+    const int t = sub * 32 + lane;
+    const int64_t row0 = int64_t(blockIdx.x) * (RT * TILES);
 
     if (threadIdx.x == 0) {
-        for (int t = 0; t <= TILES; ++t) mbar_init(&bars[t], 1);
+        for (int k = 0; k <= TILES; ++k) mbar_init(&bars[k], 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bars[0], 2 * row_bytes);
         bulk_load(s_par, weight, row_bytes, &bars[0]);
         bulk_load(s_par + row_bytes, bias, row_bytes, &bars[0]);
-        for (int t = 0; t < TILES; ++t) {
-            const int64_t r = row0 + int64_t(t) * NW;
+        for (int k = 0; k < TILES; ++k) {
+            const int64_t r = row0 + int64_t(k) * RT;
             if (r < N) {
-                const uint32_t bytes = uint32_t(min64(NW, N - r)) * row_bytes;
-                mbar_arrive_expect_tx(&bars[1 + t], bytes);
-                bulk_load(s_tiles + size_t(t) * NW * row_bytes,
+                const uint32_t bytes = uint32_t(min64(RT, N - r)) * row_bytes;
+                mbar_arrive_expect_tx(&bars[1 + k], bytes);
+                bulk_load(s_tiles + size_t(k) * RT * row_bytes,
                           reinterpret_cast<const unsigned char *>(inp) + r * row_bytes, bytes,
-                          &bars[1 + t]);
+                          &bars[1 + k]);
             }
         }
     }
@@ -103,37 +120,33 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     // they are used, so nothing row-invariant occupies registers
     const uint4 *ws = reinterpret_cast<const uint4 *>(s_par);
     const uint4 *bs = reinterpret_cast<const uint4 *>(s_par + row_bytes);
-    bool ok = tile_wait(&bars[0], status, kStatusWaitFull);
+    // A warp whose wait runs out records it; with W > 1 it still follows its
+    // row's exchanges (on meaningless data) so that the row's warps leave
+    // together.
+    bool abort = !tile_wait(&bars[0], status, kStatusWaitFull);
+    int parity = 0;
 #pragma unroll 1
-    for (int t = 0; t < TILES && ok; ++t) {
-        const int64_t r = row0 + int64_t(t) * NW + warp;
-        if (r >= N) break;                                    // warp-uniform
-        if (!tile_wait(&bars[1 + t], status, kStatusWaitFull)) {
-            ok = false;
-            break;
-        }
-        const uint4 *src =
-            reinterpret_cast<const uint4 *>(s_tiles + (size_t(t) * NW + warp) * row_bytes);
+    for (int k = 0; k < TILES; ++k) {
+        if (abort && W == 1) break;
+        const int64_t r = row0 + int64_t(k) * RT + group;
+        if (r >= N) break;                                    // uniform over the row group
+        if (!tile_wait(&bars[1 + k], status, kStatusWaitFull)) abort = true;
+        if (abort && W == 1) break;
+        const unsigned char *row = s_tiles + (size_t(k) * RT + group) * row_bytes;
+        const uint4 *src = reinterpret_cast<const uint4 *>(row);
         uint4 xv[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int j = lane + 32 * i;
+            const int j = t + TPR * i;
             xv[i] = j < nvec ? src[j] : make_uint4(0u, 0u, 0u, 0u);
         }
-        float pivot;
-        {
-            float lo, hi;
-            f32x2 p0[P];
-            to_pairs(xv[0], p0);
-            split(p0[0], lo, hi);
-            pivot = __shfl_sync(0xffffffffu, lo, 0);
-        }
+        const float pivot = to_f32(reinterpret_cast<const T *>(row)[0]);
         const f32x2 K = pair(pivot, pivot);
         f32x2 d[V][P];
         f32x2 acc = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const bool in = lane + 32 * i < nvec;
+            const bool in = t + TPR * i < nvec;
             to_pairs(xv[i], d[i]);
 #pragma unroll
             for (int q = 0; q < P; ++q) {
@@ -141,24 +154,32 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
                 if (in) acc = add2(acc, d[i][q]);
             }
         }
-        const float mean_d = warp_sum(hsum(acc)) * inv_C;
+        float sum = warp_sum(hsum(acc)), unused = 0.f;
+        abort = group_exchange<W>(sum, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                                  group, sub, lane);
+        parity ^= 1;
+        const float mean_d = sum * inv_C;
         const f32x2 M = pair(mean_d, mean_d);
         f32x2 sq = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const bool in = lane + 32 * i < nvec;
+            const bool in = t + TPR * i < nvec;
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 d[i][q] = sub2(d[i][q], M);
                 if (in) sq = fma2(d[i][q], d[i][q], sq);
             }
         }
-        const float rs = rsqrtf(warp_sum(hsum(sq)) * inv_C + eps);
+        float var = warp_sum(hsum(sq));
+        abort = group_exchange<W>(var, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                                  group, sub, lane);
+        parity ^= 1;
+        const float rs = rsqrtf(var * inv_C + eps);
         const f32x2 R = pair(rs, rs);
         uint4 *yr = reinterpret_cast<uint4 *>(out) + r * nvec;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int j = lane + 32 * i;
+            const int j = t + TPR * i;
             if (j < nvec) {
                 f32x2 wp[P], bp[P], o[P];
                 to_pairs(ws[j], wp);
@@ -168,17 +189,18 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
                 __stcs(yr + j, from_pairs(o));
             }
         }
-        if (lane == 0) {
+        if (t == 0) {
             mean[r] = pivot + mean_d;
             rstd[r] = rs;
         }
+        if (abort) break;                                     // the row group leaves together
     }
     // No block may exit while one of its copies still writes shared memory:
     // after a timeout, thread 0 waits (bounded) for every copy it issued.
-    if (!__syncthreads_and(ok) && threadIdx.x == 0) {
-        for (int t = 0; t <= TILES; ++t) {
-            if (t > 0 && row0 + int64_t(t - 1) * NW >= N) break;
-            if (!mbar_wait(&bars[t], 0)) atomicOr(status, kStatusDrain);
+    if (!__syncthreads_and(!abort) && threadIdx.x == 0) {
+        for (int k = 0; k <= TILES; ++k) {
+            if (k > 0 && row0 + int64_t(k - 1) * RT >= N) break;
+            if (!mbar_wait(&bars[k], 0)) atomicOr(status, kStatusDrain);
         }
     }
 }

@@ -108,15 +108,22 @@ template <typename T, int NC, int S>
 __host__ __device__ constexpr size_t fwd_tma_smem(int C) {
     return tma_ring_offset<T>(C, 2) + size_t(S) * NC * C * sizeof(T);
 }
-template <typename T, int NC, int S>
+template <typename T, int NC, int S, int W>
+__host__ __device__ constexpr size_t bwd_tma_ring_bytes(int C) {
+    // the ring (NC/W rows of inp and dout per stage), also reused for the
+    // end-of-block combine: at most half the row groups (rounded up) park
+    // 2C floats each
+    const size_t ring = size_t(S) * (NC / W) * 2 * C * sizeof(T);
+    const size_t comb = size_t((NC / W + 1) / 2) * 2 * C * 4;
+    return ring > comb ? ring : comb;
+}
+template <typename T, int NC, int S, int W = 1>
 __host__ __device__ constexpr size_t bwd_tma_smem(int C) {
     // weight as fp32 (read twice per row: unpacking bf16 there costs more
-    // issue slots than the wider shared-memory reads); the ring is reused for
-    // the end-of-block combine: at most NC/2 parked warps (rounded up) of 2C
-    // floats each
-    const size_t ring = size_t(S) * NC * 2 * C * sizeof(T);
-    const size_t comb = size_t((NC + 1) / 2) * 2 * C * 4;
-    return tma_ring_offset<T>(C, 1) + (ring > comb ? ring : comb);
+    // issue slots than the wider shared-memory reads), the ring, and the
+    // row-group exchange slots when rows are shared by W > 1 warps
+    return tma_ring_offset<T>(C, 1) + align128(bwd_tma_ring_bytes<T, NC, S, W>(C)) +
+           (W > 1 ? size_t(NC / W) * 2 * 3 * W * 4 : 0);
 }
 
 // Producer side, shared by both kernels: stream tiles k = 0, 1, ... of this
@@ -280,17 +287,50 @@ ln_fwd_tma_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
 }
 
 // ---------------------------------------------------------------------------
-// Backward.  Tile = NC consecutive rows (NC = 15 by default: with the
-// producer warp a 512-thread block, one per SM, 128 registers per thread);
-// block b owns tiles
-// [b*tiles_per_block, (b+1)*tiles_per_block).  A stage holds the tile's inp
-// rows followed by its dout rows.  Consumer warp w takes row w of each tile,
-// keeps dout*xhat and dout for its own columns in registers, and at the end
-// the NC warps are added in a fixed tree (as in the register-resident
-// kernel) and warp 0 writes the block's partial row.  mean/rstd of the next
+// Row-group exchange for rows shared by W warps: each warp posts its partial
+// sums (a, b) and an abort flag into a slot of its group, the group meets at a
+// named barrier, and every warp reads all W entries in the same order.  Slots
+// alternate by parity, so a slot is rewritten only after every warp of the
+// group has passed the next barrier (and so has read it).
+template <int W>
+__device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, float *slot,
+                                               int group, int sub, int lane) {
+    if constexpr (W == 1) {
+        return abort;
+    } else {
+        if (lane == 0) {
+            slot[3 * sub + 0] = a;
+            slot[3 * sub + 1] = b;
+            slot[3 * sub + 2] = abort ? 1.f : 0.f;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(group + 1), "r"(32 * W) : "memory");
+        a = 0.f;
+        b = 0.f;
+        float any = 0.f;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            a += slot[3 * k + 0];
+            b += slot[3 * k + 1];
+            any += slot[3 * k + 2];
+        }
+        return any != 0.f;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Backward.  NC consumer warps (15 by default: with the producer warp a
+// 512-thread block, one per SM, 128 registers per thread), W warps per row,
+// so a tile holds RT = NC / W consecutive rows; tiles go round-robin over
+// the persistent grid (RR) or in contiguous ranges.  A stage holds the tile's
+// inp rows followed by its dout rows.  Warp w serves row w / W of each tile
+// and, within it, vectors j = (w % W) * 32 + lane + i * 32 * W; it keeps
+// dout*xhat and dout for those columns in registers.  Row sums of the W warps
+// of a row meet in shared memory (group_exchange).  At the end the RT row
+// groups are added in a fixed tree (warps owning the same columns only) and
+// the warps of group 0 write the block's partial row.  mean/rstd of the next
 // row are prefetched one tile ahead.
 // ---------------------------------------------------------------------------
-template <typename T, int V, int NC, int S, bool RR>
+template <typename T, int V, int NC, int S, bool RR, int W = 1>
 __global__ void __launch_bounds__(32 * (NC + 1), (NC + 1) * 32 <= 256 ? 2 : 1)
 ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ dout, const T *__restrict__ inp,
@@ -298,9 +338,11 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                   int64_t tiles_per_block, unsigned *__restrict__ status) {
     static_assert(S >= 2 && S <= 8, "ring depth");
-    static_assert(NC >= 2 && NC <= 16, "consumer warps");
+    static_assert(NC % W == 0 && NC / W >= 2 && NC / W <= 15, "row groups");
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
+    constexpr int RT = NC / W;                               // rows per tile
+    constexpr int TPR = 32 * W;                              // threads per row
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + S;
@@ -308,10 +350,15 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     unsigned char *ring = smem + tma_ring_offset<T>(C, 1);
     const int nvec = C / E;
     const uint32_t row_bytes = uint32_t(C) * sizeof(T);
-    const uint32_t half_bytes = NC * row_bytes;          // inp part of a stage
+    const uint32_t half_bytes = RT * row_bytes;              // inp part of a stage
     const uint32_t stage_bytes = 2 * half_bytes;
+    float *s_red = reinterpret_cast<float *>(
+        ring + align128(bwd_tma_ring_bytes<T, NC, S, W>(C)));   // [RT][2][3W] (W > 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int group = warp / W;                              // row in the tile
+    const int sub = warp - group * W;
+    const int t = sub * 32 + lane;                           // thread within its row
 
     pdl_launch_dependents();
 
@@ -329,7 +376,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     // so that the blocks in flight cover one compact window of memory;
     // otherwise a contiguous range of tiles_per_block tiles.  Either is a
     // fixed assignment, so the column sums stay deterministic.
-    const int64_t ntiles = (N + NC - 1) / NC;
+    const int64_t ntiles = (N + RT - 1) / RT;
     const int64_t tile0 = RR ? int64_t(blockIdx.x) : int64_t(blockIdx.x) * tiles_per_block;
     const int64_t tstep = RR ? int64_t(gridDim.x) : 1;
     const int64_t ntiles_here =
@@ -350,8 +397,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             tma_produce<S>(
                 full, empty, ntiles_here, status, [&](int64_t k) { return tile0 + k * tstep; },
                 [&](int64_t tile, int st, uint64_t *bar) {
-                    const int64_t row0 = tile * NC;
-                    const uint32_t bytes = uint32_t(min64(NC, N - row0)) * row_bytes;
+                    const int64_t row0 = tile * RT;
+                    const uint32_t bytes = uint32_t(min64(RT, N - row0)) * row_bytes;
                     mbar_arrive_expect_tx(bar, 2 * bytes);
                     unsigned char *dst = ring + size_t(st) * stage_bytes;
                     bulk_load(dst, reinterpret_cast<const unsigned char *>(inp) + row0 * row_bytes,
@@ -362,32 +409,37 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 });
         }
     } else {
-        const int64_t rstep = tstep * NC;
-        int64_t r = tile0 * NC + warp;
+        const int64_t rstep = tstep * RT;
+        int64_t r = tile0 * RT + group;
         float m_next = 0.f, s_next = 0.f;
         if (ntiles_here > 0 && r < N) {
             m_next = __ldg(mean + r);
             s_next = __ldg(rstd + r);
         }
+        int parity = 0;
         for (int64_t k = 0; k < ntiles_here; ++k, r += rstep) {
             const int st = int(k % S);
-            if (!mbar_wait(&full[st], uint32_t((k / S) & 1))) {
+            // A warp whose wait runs out records it and, when it shares its
+            // row with other warps, still follows the row's exchange (with
+            // meaningless data) so that the group leaves together.
+            bool abort = !mbar_wait(&full[st], uint32_t((k / S) & 1));
+            if (abort) {
                 if (lane == 0) atomicOr(status, kStatusWaitFull);
-                break;
+                if constexpr (W == 1) break;
             }
-            const bool valid = r < N;                 // warp-uniform
+            const bool valid = r < N;                 // uniform over the row group
             const float m = m_next, s = s_next;
             if (k + 1 < ntiles_here && r + rstep < N) {   // next row's statistics
                 m_next = __ldg(mean + r + rstep);
                 s_next = __ldg(rstd + r + rstep);
             }
-            const unsigned char *stage = ring + size_t(st) * stage_bytes + warp * row_bytes;
+            const unsigned char *stage = ring + size_t(st) * stage_bytes + group * row_bytes;
             const uint4 *xs = reinterpret_cast<const uint4 *>(stage);
             const uint4 *ds = reinterpret_cast<const uint4 *>(stage + half_bytes);
             uint4 xv[V], dv[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int j = lane + 32 * i;
+                const int j = t + TPR * i;
                 const bool ok = valid && j < nvec;
                 xv[i] = ok ? xs[j] : make_uint4(0u, 0u, 0u, 0u);
                 dv[i] = ok ? ds[j] : make_uint4(0u, 0u, 0u, 0u);
@@ -396,6 +448,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
             if (!valid) continue;
+            float *slot = s_red + (group * 2 + parity) * 3 * W;
+            parity ^= 1;
 
             // Pass 1 / pass 2.  Where the register budget allows (KEEP_D), pass 1
             // keeps d = x - mean as fp32 pairs and pass 2 evaluates
@@ -405,131 +459,97 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             // xhat from the packed row.
             constexpr bool KEEP_D = sizeof(T) == 4 || V <= 3;
             uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
-            if constexpr (KEEP_D) {
-                // Pass 1: d = x - mean, g = dout * w, S1 = sum g,
-                // S2' = sum g * d (= sum g * xhat / rstd).  d stays in registers as
-                // fp32 pairs for pass 2 when that fits in the register budget
-                // (KEEP_D); otherwise pass 2 recomputes it from the packed row.
-                const f32x2 M = pair(m, m);
-                const f32x2 Sx = pair(s, s);
-                f32x2 d[V][P];
-                f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
+            const f32x2 M = pair(m, m);
+            const f32x2 Sx = pair(s, s);
+            f32x2 d[KEEP_D ? V : 1][P];
+            f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const int j = lane + 32 * i;
+            for (int i = 0; i < V; ++i) {
+                const int j = t + TPR * i;
+                if constexpr (KEEP_D) {
+                    // d for every slot (dead lanes' values are never used)
                     f32x2 dq[P];
                     to_pairs(xv[i], dq);
 #pragma unroll
-                    for (int q = 0; q < P; ++q) {
-                        dq[q] = sub2(dq[q], M);
-                        d[i][q] = dq[q];
-                    }
-                    if (j < nvec) {
-                        f32x2 dy[P], wp[P];
-                        to_pairs(dv[i], dy);
-                        smem_pairs<P>(s_w + j * E, wp);
+                    for (int q = 0; q < P; ++q) d[i][q] = sub2(dq[q], M);
+                }
+                if (j < nvec) {
+                    f32x2 dy[P], wp[P];
+                    to_pairs(dv[i], dy);
+                    smem_pairs<P>(s_w + j * E, wp);
+                    if constexpr (KEEP_D) {
 #pragma unroll
                         for (int q = 0; q < P; ++q) {
                             const f32x2 g = mul2(dy[q], wp[q]);
                             s1 = add2(s1, g);
-                            s2 = fma2(g, dq[q], s2);
+                            s2 = fma2(g, d[i][q], s2);            // sum g * d
                         }
-                    }
-                }
-                float a = hsum(s1), b = hsum(s2);
-                warp_sum2(a, b);
-                // dinp = rstd*(g - mean(g) - xhat*mean(g*xhat))
-                //      = g*rstd + NA + d*NC,  NA = -rstd*mean(g),
-                //        NC = -rstd^3 * mean(g*d)   (xhat = d*rstd)
-                const float na = -s * (a * inv_C);
-                const float nc = -(s * s) * (s * (b * inv_C));
-                const f32x2 NA = pair(na, na);
-                const f32x2 NCc = pair(nc, nc);
-#pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const int j = lane + 32 * i;
-                    if (j < nvec) {
-                        f32x2 wp[P], o[P];
-                        smem_pairs<P>(s_w + j * E, wp);
-#pragma unroll
-                        for (int q = 0; q < P; ++q) {
-                            const f32x2 dd = d[i][q];
-                            const f32x2 dy = pair_at<T>(dv[i], q);
-                            const f32x2 g = mul2(dy, wp[q]);
-                            o[q] = fma2(g, Sx, fma2(dd, NCc, NA));
-                            const f32x2 xh = mul2(dd, Sx);
-                            acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
-                            acc_b[i][q] = add2(acc_b[i][q], dy);
-                        }
-                        __stcs(gr + j, from_pairs(o));
-                    }
-                }
-            } else {
-                const f32x2 M = pair(m, m);
-                const f32x2 Sx = pair(s, s);
-                f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
-#pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const int j = lane + 32 * i;
-                    if (j < nvec) {
-                        f32x2 x[P], dy[P], wp[P];
+                    } else {
+                        f32x2 x[P];
                         to_pairs(xv[i], x);
-                        to_pairs(dv[i], dy);
-                        smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
                         for (int q = 0; q < P; ++q) {
                             const f32x2 xh = mul2(sub2(x[q], M), Sx);
                             const f32x2 g = mul2(dy[q], wp[q]);
                             s1 = add2(s1, g);
-                            s2 = fma2(g, xh, s2);
+                            s2 = fma2(g, xh, s2);                 // sum g * xhat
                         }
-                    }
-                }
-                float a = hsum(s1), b = hsum(s2);
-                warp_sum2(a, b);
-                const float na = -s * (a * inv_C);
-                const float nc = -s * (b * inv_C);
-                const f32x2 NA = pair(na, na);
-                const f32x2 NCc = pair(nc, nc);
-#pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const int j = lane + 32 * i;
-                    if (j < nvec) {
-                        f32x2 x[P], dy[P], wp[P], o[P];
-                        to_pairs(xv[i], x);
-                        to_pairs(dv[i], dy);
-                        smem_pairs<P>(s_w + j * E, wp);
-#pragma unroll
-                        for (int q = 0; q < P; ++q) {
-                            const f32x2 xh = mul2(sub2(x[q], M), Sx);
-                            const f32x2 g = mul2(dy[q], wp[q]);
-                            o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
-                            acc_w[i][q] = fma2(dy[q], xh, acc_w[i][q]);
-                            acc_b[i][q] = add2(acc_b[i][q], dy[q]);
-                        }
-                        __stcs(gr + j, from_pairs(o));
                     }
                 }
             }
+            float a = hsum(s1), b = hsum(s2);
+            warp_sum2(a, b);
+            abort = group_exchange<W>(a, b, abort, slot, group, sub, lane);
+            const float na = -s * (a * inv_C);
+            const float nc = KEEP_D ? -(s * s) * (s * (b * inv_C)) : -s * (b * inv_C);
+            const f32x2 NA = pair(na, na);
+            const f32x2 NCc = pair(nc, nc);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = t + TPR * i;
+                if (j < nvec) {
+                    f32x2 wp[P], o[P];
+                    smem_pairs<P>(s_w + j * E, wp);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        const f32x2 dy = pair_at<T>(dv[i], q);
+                        const f32x2 g = mul2(dy, wp[q]);
+                        f32x2 xh;
+                        if constexpr (KEEP_D) {
+                            o[q] = fma2(g, Sx, fma2(d[i][q], NCc, NA));
+                            xh = mul2(d[i][q], Sx);
+                        } else {
+                            xh = mul2(sub2(pair_at<T>(xv[i], q), M), Sx);
+                            o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
+                        }
+                        acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
+                        acc_b[i][q] = add2(acc_b[i][q], dy);
+                    }
+                    __stcs(gr + j, from_pairs(o));
+                }
+            }
+            if (abort) break;                         // the whole row group leaves here
         }
     }
 
-    // Fixed-order tree over the NC consumer warps: at each level with width h
-    // (the largest power of two below the active count n, then halving),
-    // warps [h, n) park their sums and warps [0, n - h) add them.  The ring
-    // is free again once every warp has passed the first barrier (all copies
-    // were consumed, or drained by the producer).
+    // Fixed-order tree over the RT row groups (warps owning the same columns
+    // only): at each level with width h (the largest power of two below the
+    // active count n, then halving), groups [h, n) park their sums and groups
+    // [0, n - h) add them.  The ring is free again once every warp has
+    // passed the first barrier (all copies were consumed, or drained by the
+    // producer).
     __syncthreads();
     float *s_acc = reinterpret_cast<float *>(ring);
-    constexpr int kTop = (NC > 8) ? 8 : (NC > 4) ? 4 : (NC > 2) ? 2 : 1;
-    int n = NC;
+    constexpr int kTop = (RT > 8) ? 8 : (RT > 4) ? 4 : (RT > 2) ? 2 : 1;
+    const bool consumer = warp < NC;
+    int n = RT;
 #pragma unroll
     for (int h = kTop; h >= 1; h /= 2) {
-        if (warp >= h && warp < n) {
-            float *dst = s_acc + (warp - h) * 2 * C;
+        if (consumer && group >= h && group < n) {
+            float *dst = s_acc + (group - h) * 2 * C;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int j = lane + 32 * i;
+                const int j = t + TPR * i;
                 if (j < nvec) {
                     ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(dst + j * E);
                     ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(dst + C + j * E);
@@ -542,11 +562,11 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             }
         }
         __syncthreads();
-        if (warp < n - h) {
-            const float *src = s_acc + warp * 2 * C;
+        if (consumer && group < n - h) {
+            const float *src = s_acc + group * 2 * C;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int j = lane + 32 * i;
+                const int j = t + TPR * i;
                 if (j < nvec) {
                     f32x2 pw[P], pb[P];
                     smem_pairs<P>(src + j * E, pw);
@@ -562,11 +582,11 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
         __syncthreads();
         n = h;
     }
-    if (warp == 0) {
+    if (consumer && group == 0) {
         float *pblk = partial + (int64_t)blockIdx.x * 2 * C;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int j = lane + 32 * i;
+            const int j = t + TPR * i;
             if (j < nvec) {
                 ulonglong2 *pw = reinterpret_cast<ulonglong2 *>(pblk + j * E);
                 ulonglong2 *pb = reinterpret_cast<ulonglong2 *>(pblk + C + j * E);
