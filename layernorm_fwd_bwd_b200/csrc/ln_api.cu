@@ -126,13 +126,15 @@ cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t st
     cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    // Every kernel here starts with pdl_enter() (griddepcontrol.wait before
+    // any global memory access), so programmatic serialization is always
+    // safe; `pdl` is kept for call-site readability.
+    (void)pdl;
     cudaLaunchAttribute attr[1];
-    if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
     if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
     return e;
@@ -147,13 +149,15 @@ cudaError_t launch_cluster(K kernel, int grid, int threads, size_t smem, cudaStr
     cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
     if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
     return e;
@@ -436,18 +440,18 @@ struct BwdVec {
                 return;
             }
         }
-        if constexpr ((W == 1 || W == 2) && LN_BWD_STYLE >= 1) {
-            constexpr int NC = lnk::BwdRingConsumers<W>::value;
-            constexpr int S = lnk::BwdStages<V, NC>::value;
-            constexpr int RT = NC / W;                    // rows per tile
-            status = bwd_run<T, true>(
-                a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
-                lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
-        } else {
-            status = bwd_run<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
-                                       32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
-                                       GROUPS, 1);
-        }
+        status = bwd_run<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
+                                   32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
+                                   GROUPS, 1);
+    }
+    template <int V, int W>
+    void ring() {
+        constexpr int NC = lnk::BwdRingConsumers<W>::value;
+        constexpr int S = lnk::BwdStages<V, NC>::value;
+        constexpr int RT = NC / W;                        // rows per tile
+        status = bwd_run<T, true>(
+            a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
+            lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
     }
 };
 
@@ -464,6 +468,7 @@ int bwd_dispatch(const BwdArgs &a) {
                         aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
     if (vec_ok) {
         BwdVec<T> v{a};
+        if (LN_BWD_STYLE == 1 && lnk::visit_bwd_ring<T>(a.C / E, v)) return v.status;
         if (lnk::visit_bwd_vec<T>(a.C / E, v)) return v.status;
     }
     return bwd_scalar<T>(a);

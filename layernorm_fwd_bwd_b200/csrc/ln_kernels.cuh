@@ -168,14 +168,16 @@ __device__ __forceinline__ void block_sum2(float &a, float &b, float *slot, int 
     }
 }
 
-// Programmatic dependent launch (sm_90+): let the next grid on the stream be
-// scheduled now / wait until the previous grid has completed and its writes
-// are visible.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait_primary() {
+// Programmatic dependent launch (sm_90+).  Every kernel of this library is
+// launched with programmatic stream serialization and starts with
+// pdl_enter(): it first waits until the previous grid on the stream has
+// completed and its writes are visible (so stream order holds for every
+// global memory access that follows), then allows the next grid to be
+// scheduled.  What overlaps is only the launch and block scheduling of the
+// next kernel with the tail of the current one.
+__device__ __forceinline__ void pdl_enter() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -350,6 +352,7 @@ __global__ void __launch_bounds__(32 * W * GROUPS)
 ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                   const T *__restrict__ inp, const T *__restrict__ weight,
                   const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps) {
+    pdl_enter();
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
@@ -457,6 +460,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ weight, const float *__restrict__ mean,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                   int64_t rows_per_block) {
+    pdl_enter();
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
@@ -466,7 +470,6 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     float *s_acc = s_w + C;                                   // [GROUPS/2][2C]
     float *s_red0 = s_acc + (GROUPS > 1 ? (GROUPS / 2) * 2 * C : 0);
 
-    pdl_launch_dependents();
 
     for (int c = threadIdx.x; c < C; c += blockDim.x) s_w[c] = to_f32(weight[c]);
     __syncthreads();
@@ -630,8 +633,8 @@ constexpr int kColsumThreads = 1024;
 static __global__ void __launch_bounds__(kColsumThreads)
 ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
                  const float *__restrict__ partial, int G, int C) {
+    pdl_enter();
     constexpr int S = kColsumThreads / 32;
-    pdl_wait_primary();
     __shared__ float s[S][33];
     const int tx = threadIdx.x & 31;
     const int ty = threadIdx.x >> 5;
@@ -674,6 +677,7 @@ ln_fwd_scalar_kernel(T *__restrict__ out, float *__restrict__ mean,
                      float *__restrict__ rstd, const T *__restrict__ inp,
                      const T *__restrict__ weight, const T *__restrict__ bias, int64_t N,
                      int C, float inv_C, float eps) {
+    pdl_enter();
     __shared__ float s_red[2][32];
     const int tpr = BLOCK_ROW ? (int)blockDim.x : 32;
     const int groups = blockDim.x / tpr;
@@ -718,8 +722,8 @@ ln_bwd_scalar_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                      const T *__restrict__ weight, const float *__restrict__ mean,
                      const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                      int64_t rows_per_block) {
+    pdl_enter();
     __shared__ float s_red[2][64];
-    pdl_launch_dependents();
     const int tpr = blockDim.x;
     const int nwarps = tpr >> 5;
     float *pw = partial + (int64_t)blockIdx.x * 2 * C;

@@ -94,13 +94,15 @@ cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t st
     cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    // Every kernel here starts with pdl_enter() (griddepcontrol.wait before
+    // any global memory access), so programmatic serialization is always
+    // safe; `pdl` is kept for call-site readability.
+    (void)pdl;
     cudaLaunchAttribute attr[1];
-    if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
     if (e == cudaSuccess) ln_internal_count_launches(1);
     return e;
@@ -205,18 +207,18 @@ struct Vec {
                 return;
             }
         }
-        if constexpr ((W == 1 || W == 2) && LN_BWD_STYLE >= 1) {
-            constexpr int NC = lnk::BwdRingConsumers<W>::value;
-            constexpr int S = lnk::BwdStages<V, NC>::value;
-            constexpr int RT = NC / W;                    // rows per tile
-            status = run_kernel<T, true>(
-                a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
-                lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
-        } else {
-            status = run_kernel<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
-                                          32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
-                                          GROUPS, 1);
-        }
+        status = run_kernel<T, false>(a, lnk::ln_bwd_vec_kernel<T, V, W, GROUPS>,
+                                      32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
+                                      GROUPS, 1);
+    }
+    template <int V, int W>
+    void ring() {
+        constexpr int NC = lnk::BwdRingConsumers<W>::value;
+        constexpr int S = lnk::BwdStages<V, NC>::value;
+        constexpr int RT = NC / W;                        // rows per tile
+        status = run_kernel<T, true>(
+            a, lnk::ln_bwd_tma_kernel<T, V, NC, S, LN_BWD_RING_RR != 0, W>, 32 * (NC + 1),
+            lnk::bwd_tma_smem<T, NC, S, W>(a.C), RT, RT);
     }
 };
 
@@ -229,6 +231,7 @@ int dispatch(const Args &a) {
                         aligned16(a.dout) && aligned16(a.inp) && aligned16(a.weight);
     if (vec_ok) {
         Vec<T> v{a};
+        if (LN_BWD_STYLE == 1 && lnk::visit_bwd_ring<T>(a.C / E, v)) return v.status;
         if (lnk::visit_bwd_vec<T>(a.C / E, v)) return v.status;
     }
     const int threads = (int)std::min<int64_t>(512, ceil_div(a.C, 32) * 32);

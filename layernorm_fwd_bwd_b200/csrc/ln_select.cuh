@@ -117,6 +117,42 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
     return false;
 }
 
+// Backward ring (ln_tma.cuh).  One warp per row while a lane holds at most
+// 4 (bf16) / 6 (fp32) vectors; wider rows are split over W = 2..4 warps with
+// 3 (bf16) / 5 (fp32) vectors per lane, which keeps x - mean in registers
+// between the two passes.  Measured on B200: bf16 C = 1024 is faster on one
+// warp (4 vectors, recomputing x - mean) than on two (the row-group exchange
+// costs more than it saves); C = 1600 is faster on three warps (43 us) than
+// on two with 4 vectors (46 us).  Calls visitor.template ring<V, W>();
+// false when rows are wider than 4 warps cover.
+template <typename T> struct RingVmax { static constexpr int one = 6, shared = 5; };
+template <> struct RingVmax<bf16> { static constexpr int one = 4, shared = 3; };
+
+template <typename T, typename Visitor>
+bool visit_bwd_ring(int nvec, Visitor &v) {
+    constexpr int V1 = RingVmax<T>::one;
+    constexpr int VS = RingVmax<T>::shared;
+    const int v1 = (nvec + 31) / 32;
+    switch (v1) {
+        case 1: v.template ring<1, 1>(); return true;
+        case 2: v.template ring<2, 1>(); return true;
+        case 3: v.template ring<3, 1>(); return true;
+        case 4: v.template ring<4, 1>(); return true;
+        default: break;
+    }
+    if constexpr (V1 > 4) {
+        if (v1 == 5) { v.template ring<5, 1>(); return true; }
+        if (v1 == 6) { v.template ring<6, 1>(); return true; }
+    }
+    const int w = (nvec + 32 * VS - 1) / (32 * VS);          // warps per row at VS
+    switch (w) {
+        case 2: v.template ring<VS, 2>(); return true;
+        case 3: v.template ring<VS, 3>(); return true;
+        case 4: v.template ring<VS, 4>(); return true;
+        default: return false;
+    }
+}
+
 template <typename T, typename Visitor>
 bool visit_bwd_vec(int nvec, Visitor &v) {
     constexpr int VM = BwdVmaxW1<T>::value;

@@ -76,6 +76,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
                    const T *__restrict__ inp, const T *__restrict__ weight,
                    const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps,
                    unsigned *__restrict__ status) {
+    pdl_enter();
     static_assert(TILES + 1 <= 16, "barriers fit in 128 bytes");
     static_assert(NW % W == 0 && NW / W <= 15, "row groups");
     constexpr int E = Vec<T>::E;
@@ -218,6 +219,7 @@ ln_bwd_tile_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                    const T *__restrict__ weight, const float *__restrict__ mean,
                    const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                    unsigned *__restrict__ status) {
+    pdl_enter();
     static_assert(TILES + 1 <= 16, "barriers fit in 128 bytes");
     static_assert(NW >= 2 && NW <= 16, "warps per block");
     namespace cg = cooperative_groups;
@@ -236,7 +238,6 @@ ln_bwd_tile_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     const size_t tile_bytes = size_t(NW) * row_bytes;         // one array of one tile
     const bool has_rows = row0 < N;                           // false: cluster padding
 
-    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int t = 0; t <= TILES; ++t) mbar_init(&bars[t], 1);

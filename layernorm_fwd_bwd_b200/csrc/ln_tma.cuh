@@ -161,6 +161,7 @@ ln_fwd_tma_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
                   const T *__restrict__ inp, const T *__restrict__ weight,
                   const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps,
                   unsigned *__restrict__ status) {
+    pdl_enter();
     static_assert(S >= 2 && S <= 8, "ring depth");
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
@@ -337,6 +338,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ weight, const float *__restrict__ mean,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
                   int64_t tiles_per_block, unsigned *__restrict__ status) {
+    pdl_enter();
     static_assert(S >= 2 && S <= 8, "ring depth");
     static_assert(NC % W == 0 && NC / W >= 2 && NC / W <= 15, "row groups");
     constexpr int E = Vec<T>::E;
@@ -360,7 +362,6 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     const int sub = warp - group * W;
     const int t = sub * 32 + lane;                           // thread within its row
 
-    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
