@@ -50,7 +50,7 @@ METRIC = "LayerNorm fwd+bwd GB/s and rows/s at 1 B200; % of HBM roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 SETS = 4
-EVERY = 16          # per-call events on one timed step in EVERY
+EVERY = 64          # per-call events on one timed step in EVERY
 KERNEL_SOURCES = [os.path.join(ROOT, "layernorm_fwd_bwd_b200", "csrc", f)
                   for f in ("ln_kernels.cuh", "ln_select.cuh", "ln_tma.cuh", "ln_tile.cuh",
                             "ln_api.cu")]
