@@ -257,9 +257,17 @@ struct FwdVec {
     }
     template <int V, int RW>
     void run_tile() {
+        constexpr int E = lnk::Vec<T>::E;
+        if (a.C / E == 32 * RW * V)
+            run_tile_k<V, RW, true>();
+        else
+            run_tile_k<V, RW, false>();
+    }
+    template <int V, int RW, bool FULL>
+    void run_tile_k() {
         constexpr int NW = lnk::kTileWarps * RW;          // 8 rows per tile either way
         constexpr int TL = lnk::kTileFwdTiles;
-        auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL, RW>;
+        auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL, RW, FULL>;
         const int threads = 32 * NW;
         const size_t smem = lnk::fwd_tile_smem<T, NW, TL, RW>(a.C);
         int occ = 0;

@@ -68,9 +68,9 @@ __device__ __forceinline__ bool tile_wait(uint64_t *bar, unsigned *status, unsig
 // first element, read from shared memory by every warp of the row; with
 // W > 1 the row sums meet through group_exchange (ln_tma.cuh).
 // Requirements (checked by the host): inp/out/weight/bias 16-byte aligned,
-// C * sizeof(T) a multiple of 16, C / E <= 32 * W * V.
+// C * sizeof(T) a multiple of 16, C / E <= 32 * W * V (== when FULL).
 // ---------------------------------------------------------------------------
-template <typename T, int V, int NW, int TILES, int W = 1>
+template <typename T, int V, int NW, int TILES, int W = 1, bool FULL = false>
 __global__ void __launch_bounds__(32 * NW)
 ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                    const T *__restrict__ inp, const T *__restrict__ weight,
@@ -90,7 +90,9 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     unsigned char *s_tiles = s_par + align128(size_t(2) * row_bytes);
     float *s_red = reinterpret_cast<float *>(
         s_tiles + align128(size_t(TILES) * RT * row_bytes));   // [RT][2][3W] (W > 1)
-    const int nvec = C / E;
+    // FULL: the row is exactly 32 * W * V vectors, so no lane is ever past
+    // its end and every bound check below folds away at compile time
+    const int nvec = FULL ? 32 * W * V : C / E;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int group = warp / W;
