@@ -35,6 +35,14 @@ stress_fp32_65536x768  f32    65536   768    100 + 0.01 N(0,1), every 100th row
 weight ~ 1 + 0.1 N(0,1) and bias ~ 0.1 N(0,1) everywhere; eps = 1e-5.  In the
 stress case every row r with r % 100 == 0 holds one value v_r = 100 + 0.01 z_r
 (one draw per row) in all C columns, so its variance is exactly zero.
+
+Inputs of the variants (``generate_extras``, streams of their own so the
+arrays above do not change): the residual branch added to inp by the fused
+residual forward, branch ~ N(0, inp_sigma^2) (a sub-layer output at the
+residual stream's own spread; in the stress case the sum stays near 100), a
+previous dinp for the accumulating backward, N(0, (dout_sigma /
+inp_sigma)^2) (the scale of dinp itself, rstd * dout * weight), and previous
+dweight and dbias, fp32 N(0,1).
 """
 from __future__ import annotations
 
@@ -49,6 +57,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # stream ids: one per drawn array
 S_INP, S_WEIGHT, S_BIAS, S_DOUT, S_CONST = 0, 1, 2, 3, 4
+S_BRANCH, S_DINP_PREV, S_PARAM_PREV = 5, 6, 7
 
 EPS = float(np.float32(1e-5))
 
@@ -214,3 +223,38 @@ def custom(dtype: str, N: int, C: int, seed: int, inp_mu: float = 0.0,
     w = Workload(f"custom_{dtype}_{N}x{C}", dtype, N, C, seed, inp_mu, inp_sigma,
                  dout_sigma, const_row_period)
     return generate(w)
+
+
+@dataclasses.dataclass
+class Extras:
+    """Inputs of the variants, for the same rows as a Batch."""
+    workload: Workload
+    rows: np.ndarray
+    branch: np.ndarray        # [len(rows), C] storage: added to inp (residual forward)
+    dinp_prev: np.ndarray     # [len(rows), C] storage: accumulated into (backward)
+    dweight_prev: np.ndarray  # [C] float32
+    dbias_prev: np.ndarray    # [C] float32
+
+    def f64(self, name: str) -> np.ndarray:
+        a = getattr(self, name)
+        if name in ("dweight_prev", "dbias_prev"):
+            return a.astype(np.float64)
+        return storage_to_f64(a, self.workload.dtype)
+
+
+def generate_extras(w: Workload, rows=None, chunk_rows: int = 8192) -> Extras:
+    """Draw the variants' inputs for ``rows`` (all rows when None)."""
+    rows = np.arange(w.N, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    if rows.size and (rows.min() < 0 or rows.max() >= w.N):
+        raise ValueError("row index out of range")
+    store = np.float32 if w.dtype == F32 else np.uint16
+    branch = np.empty((rows.size, w.C), store)
+    prev = np.empty((rows.size, w.C), store)
+    for a in range(0, rows.size, chunk_rows):
+        rr = rows[a:a + chunk_rows]
+        branch[a:a + rr.size] = to_storage(_rows_block(w, rr, S_BRANCH, 0.0, w.inp_sigma), w.dtype)
+        prev[a:a + rr.size] = to_storage(
+            _rows_block(w, rr, S_DINP_PREV, 0.0, w.dout_sigma / w.inp_sigma), w.dtype)
+    cidx = np.arange(2 * w.C, dtype=np.uint64)
+    params = normals(w.seed, S_PARAM_PREV, cidx).astype(np.float32)
+    return Extras(w, rows, branch, prev, params[:w.C].copy(), params[w.C:].copy())

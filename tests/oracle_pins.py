@@ -18,7 +18,17 @@ What pins what:
               L = sum(out * dout) through the forward, the per-row identities
               sum_c dinp = 0 and sum_c dinp * xhat = rstd * eps/(var+eps) *
               sum_c g * xhat, exact integer column sums for dbias, hand-worked
-              examples, and torch autograd in float64.
+              examples, and torch autograd in float64;
+  rounding -- brute force: every finite value of bfloat16 and fp16 (and the
+              fp32 values near each probe) enumerated from its bit pattern,
+              the nearest chosen with exact rational arithmetic, ties to the
+              even bit pattern; numpy's float32 and float16 casts;
+  residual forward -- the rounded sum against that brute force on the exact
+              (rational) sum, and branch = 0 reducing to the plain forward;
+  backward variants -- linearity of the gradient in dout (accumulating the
+              gradient of dout1 into that of dout2 gives the gradient of
+              dout1 + dout2) and torch autograd in float64, which computes the
+              statistics itself (the recomputing variant).
 """
 from __future__ import annotations
 
@@ -318,7 +328,165 @@ def pin_rejects_bad_shapes(orc):
     assert np.array_equal(dw, np.zeros(4)) and np.array_equal(db, np.zeros(4))
 
 
+# ----------------------------------------------------------- rounding pins
+
+def _format_values(fmt):
+    """Every positive finite value of a format, ascending, with its bit
+    pattern (for fp32, only bf16 and f16 are enumerated: 2^31 values are too
+    many; fp32 is pinned by numpy's cast and by local neighbourhoods)."""
+    if fmt == "bf16":
+        bits = np.arange(1, 0x7F80, dtype=np.uint32)
+        vals = (bits << np.uint32(16)).view(np.float32).astype(np.float64)
+    elif fmt == "f16":
+        bits = np.arange(1, 0x7C00, dtype=np.uint16)
+        vals = bits.view(np.float16).astype(np.float64)
+        bits = bits.astype(np.uint32)
+    else:
+        raise ValueError(fmt)
+    return vals, bits
+
+
+def _brute_round(v, vals, bits):
+    """Nearest of 0 and ``vals`` to the exact value v (Fraction or float), ties
+    to the even bit pattern; beyond the largest value by half a spacing or
+    more, infinity."""
+    v = Fraction(v)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    top = Fraction(float(vals[-1]))
+    half_top = (top - Fraction(float(vals[-2]))) / 2
+    if a >= top + half_top:
+        return sign * math.inf
+    k = int(np.searchsorted(vals, float(a), side="right"))   # vals[k-1] <= a (about)
+    cands = [(Fraction(0), 0)]
+    for j in range(max(0, k - 2), min(len(vals), k + 2)):
+        cands.append((Fraction(float(vals[j])), int(bits[j])))
+    best = min(cands, key=lambda cb: (abs(cb[0] - a), cb[1] & 1))
+    return sign * float(best[0])
+
+
+def _probe_values(rng, lo_exp, hi_exp, n):
+    """Random magnitudes over [2^lo_exp, 2^hi_exp), both signs."""
+    e = rng.uniform(lo_exp, hi_exp, n)
+    return np.where(rng.random(n) < 0.5, -1.0, 1.0) * np.exp2(e)
+
+
+def pin_round_brute_force(orc):
+    """oracle_round_format against brute force over every bfloat16 and fp16
+    value: random values across the normal and subnormal ranges, exact ties
+    (midpoints of neighbouring values) and the overflow boundary."""
+    rng = _rng(21)
+    for fmt, (lo, hi) in (("bf16", (-136.0, 128.5)), ("f16", (-26.0, 16.5))):
+        vals, bits = _format_values(fmt)
+        probes = list(_probe_values(rng, lo, hi, 400))
+        idx = rng.integers(0, len(vals) - 1, 200)
+        probes += [float((Fraction(float(vals[i])) + Fraction(float(vals[i + 1]))) / 2)
+                   for i in idx]                                    # exact midpoints
+        top, below = float(vals[-1]), float(vals[-2])
+        probes += [top, top + (top - below) / 2, np.nextafter(top + (top - below) / 2, 0.0),
+                   float(vals[0]) / 2, float(vals[0]) * 1.5, -float(vals[0]) / 2]
+        got = orc.round_to(np.array(probes), fmt)
+        for v, g in zip(probes, got):
+            want = _brute_round(v, vals, bits)
+            assert g == want or (math.isinf(want) and g == want), \
+                f"{fmt}: round({v!r}) = {g!r}, brute force {want!r}"
+
+
+def pin_round_numpy_casts(orc):
+    """fp32 and fp16 rounding against numpy's float64 -> float32 / float16
+    casts (IEEE round to nearest even), including fp32 ties built exactly
+    as midpoints of neighbouring fp32 values and subnormals."""
+    rng = _rng(22)
+    v32 = _probe_values(rng, -155.0, 128.5, 20000)
+    f = rng.normal(size=2000).astype(np.float32)
+    mids = (f.astype(np.float64)
+            + (np.nextafter(f, np.float32(np.inf)).astype(np.float64) - f.astype(np.float64)) / 2)
+    v32 = np.concatenate([v32, mids, [3.4028235677973366e38, 3.40282357e38, 1e-46, -7e-46]])
+    with np.errstate(over="ignore"):
+        want32 = v32.astype(np.float32).astype(np.float64)
+    got32 = orc.round_to(v32, "f32")
+    assert np.array_equal(got32, want32), "fp32 rounding disagrees with numpy"
+    v16 = _probe_values(rng, -27.0, 16.5, 20000)
+    with np.errstate(over="ignore"):
+        want16 = v16.astype(np.float16).astype(np.float64)
+    assert np.array_equal(orc.round_to(v16, "f16"), want16), "fp16 rounding vs numpy"
+
+
+def pin_residual_forward(orc):
+    """forward_residual: x is the brute-force rounding of the exact sum
+    resid + branch (bf16 operands), and with branch = 0 the whole result is
+    the plain forward of resid."""
+    rng = _rng(23)
+    vals, bits = _format_values("bf16")
+    n, C = 3, 11
+    a = orc.round_to(rng.normal(size=(n, C)), "bf16")
+    b = orc.round_to(rng.normal(scale=0.3, size=(n, C)) * np.exp2(rng.integers(-12, 4, (n, C))),
+                     "bf16")
+    w = 1.0 + 0.1 * rng.normal(size=C)
+    bias = 0.1 * rng.normal(size=C)
+    x, out, mean, rstd = orc.forward_residual(a, b, w, bias, 1e-5, "bf16")
+    for i in range(n):
+        for j in range(C):
+            want = _brute_round(Fraction(float(a[i, j])) + Fraction(float(b[i, j])), vals, bits)
+            assert x[i, j] == want, "residual sum rounding"
+    o2, m2, s2 = orc.forward(x, w, bias, 1e-5)
+    assert np.array_equal(out, o2) and np.array_equal(mean, m2) and np.array_equal(rstd, s2)
+    x0, o0, m0, s0 = orc.forward_residual(a, np.zeros_like(a), w, bias, 1e-5, "bf16")
+    o1, m1, s1 = orc.forward(a, w, bias, 1e-5)
+    assert np.array_equal(x0, a), "x = resid when branch = 0"
+    assert np.array_equal(o0, o1) and np.array_equal(m0, m1) and np.array_equal(s0, s1)
+
+
+# -------------------------------------------------------- backward variants
+
+def pin_backward_linearity(orc):
+    """The gradient is linear in dout: accumulating the gradient of dout2
+    onto that of dout1 gives the gradient of dout1 + dout2 (dinp, dweight and
+    dbias), with saved and with recomputed statistics."""
+    rng = _rng(24)
+    n, C, eps = 6, 19, 1e-5
+    x = rng.normal(size=(n, C))
+    w = 1.0 + 0.1 * rng.normal(size=C)
+    d1, d2 = rng.normal(size=(n, C)), rng.normal(size=(n, C))
+    _, mean, rstd = orc.forward(x, w, np.zeros(C), eps)
+    for recompute in (False, True):
+        g1 = orc.backward_ex(d1, x, w, mean, rstd, eps, recompute=recompute)
+        acc = orc.backward_ex(d2, x, w, mean, rstd, eps, dinp_prev=g1[0], dweight_prev=g1[1],
+                              dbias_prev=g1[2], recompute=recompute)
+        both = orc.backward(d1 + d2, x, w, mean, rstd)
+        for got, want, name in zip(acc, both, ("dinp", "dweight", "dbias")):
+            assert _rel(got, want) < 1e-12, f"accumulated {name} (recompute={recompute})"
+    # accumulating only the parameters leaves dinp overwritten
+    g = orc.backward_ex(d2, x, w, mean, rstd, eps, dweight_prev=np.ones(C), dbias_prev=np.ones(C))
+    plain = orc.backward(d2, x, w, mean, rstd)
+    assert _rel(g[0], plain[0]) < 1e-15 and _rel(g[1] - 1.0, plain[1]) < 1e-12
+
+
+def pin_backward_recompute_torch(orc):
+    """Recomputing the statistics: torch autograd of layer_norm in float64
+    (which computes mean and rstd from the input itself), including rows whose
+    variance is comparable to eps."""
+    import torch
+    rng = _rng(25)
+    for (n, C, eps, mu, sig) in ((7, 33, 1e-5, 0.0, 1.0), (4, 768, 1e-5, 100.0, 0.01),
+                                 (5, 64, 1e-5, 0.0, 2e-3)):
+        x = mu + sig * rng.normal(size=(n, C))
+        w = 1.0 + 0.1 * rng.normal(size=C)
+        dout = rng.normal(size=(n, C))
+        tx = torch.tensor(x, dtype=torch.float64, requires_grad=True)
+        tw = torch.tensor(w, dtype=torch.float64, requires_grad=True)
+        tb = torch.zeros(C, dtype=torch.float64, requires_grad=True)
+        torch.nn.functional.layer_norm(tx, (C,), tw, tb, eps).backward(
+            torch.tensor(dout, dtype=torch.float64))
+        dinp, dw, db = orc.backward_ex(dout, x, w, None, None, eps, recompute=True)
+        tol = 1e-12 if sig >= 1 else 1e-9
+        assert _rel(dinp, tx.grad.numpy()) < tol, "recomputed dinp vs torch"
+        assert _rel(dw, tw.grad.numpy()) < tol, "recomputed dweight vs torch"
+        assert _rel(db, tb.grad.numpy()) < 1e-13, "recomputed dbias vs torch"
+
+
 ALL_PINS = [pin_one_column, pin_two_columns, pin_constant_rows, pin_scale_by_two,
             pin_shift_invariance, pin_unit_affine_moments, pin_finite_differences,
             pin_row_identities, pin_dbias_integer_sum, pin_hand_worked,
-            pin_torch_float64]
+            pin_torch_float64, pin_round_brute_force, pin_round_numpy_casts,
+            pin_residual_forward, pin_backward_linearity, pin_backward_recompute_torch]

@@ -30,6 +30,29 @@ MUTANTS = [
      "double xhat = (x[c] - m) / s;"),
     ("dbias_times_weight", "dbias[c] += dy[c];", "dbias[c] += dy[c] * weight[c];"),
     ("dweight_uses_g", "dweight[c] += dy[c] * xhat;", "dweight[c] += g * xhat;"),
+    # rounding to a format
+    ("round_ties_away", "nearbyint(ldexp(v, -q))", "round(ldexp(v, -q))"),
+    ("round_truncates", "nearbyint(ldexp(v, -q))", "trunc(ldexp(v, -q))"),
+    ("round_one_bit_short", "int q = e - p;", "int q = e - p + 1;"),
+    ("round_no_gradual_underflow", "if (q < emin - p + 1) q = emin - p + 1;", ""),
+    ("round_no_overflow", "fabs(r) > max_finite ? copysign(INFINITY, v) : r", "r"),
+    # residual forward
+    ("residual_drops_branch", "x[i] = resid[i] + branch[i];", "x[i] = resid[i];"),
+    ("residual_not_rounded", "int rc = oracle_round_format(x, x, N * C, p, emin, max_finite);",
+     "int rc = ORACLE_OK;"),
+    # backward variants
+    ("accumulate_dinp_ignored", "dinp[i] = accumulate_dinp ? dinp[i] + g_in[i] : g_in[i];",
+     "dinp[i] = g_in[i];"),
+    ("accumulate_dinp_subtracts", "dinp[i] = accumulate_dinp ? dinp[i] + g_in[i] : g_in[i];",
+     "dinp[i] = accumulate_dinp ? dinp[i] - g_in[i] : g_in[i];"),
+    ("accumulate_params_ignored",
+     "dweight[j] = accumulate_params ? dweight[j] + g_w[j] : g_w[j];", "dweight[j] = g_w[j];"),
+    ("accumulate_dbias_ignored",
+     "dbias[j] = accumulate_params ? dbias[j] + g_b[j] : g_b[j];", "dbias[j] = g_b[j];"),
+    ("recompute_ignored", "            m = st_m;\n            s = st_s;\n", ""),
+    ("recompute_without_eps",
+     "rc = oracle_ln_forward(scratch, st_m, st_s, inp, weight, zeros, N, C, eps);",
+     "rc = oracle_ln_forward(scratch, st_m, st_s, inp, weight, zeros, N, C, 1e-300);"),
 ]
 
 
