@@ -29,10 +29,11 @@
  * dinp, weight and bias.  mean, rstd, dweight and dbias are always fp32.
  * Arithmetic is fp32 in registers; bf16 results are rounded to nearest-even.
  *
- * Semantics shared by both calls.
+ * Semantics shared by every call.
  *   - Asynchronous on `stream` (NULL: the legacy default stream); no host
  *     synchronisation; the library creates no streams of its own.
- *   - Outputs are overwritten, never accumulated into.
+ *   - Outputs are overwritten, never accumulated into, except where
+ *     ln_backward_ex is asked to accumulate.
  *   - Results are deterministic: the same inputs give bitwise-identical
  *     outputs on every call (no floating-point atomics).
  *   - Any alignment is accepted.  Fully 16-byte-aligned arrays with C * size
@@ -76,7 +77,8 @@ typedef enum {
     LN_ERR_EPS = 4,        /* eps is not finite, or not > 0 */
     LN_ERR_WORKSPACE = 5,  /* the backward's workspace could not be allocated */
     LN_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
-    LN_ERR_SCRATCH = 7     /* ln_backward_noalloc: C > LN_NOALLOC_MAX_C */
+    LN_ERR_SCRATCH = 7,    /* ln_backward_noalloc: C > LN_NOALLOC_MAX_C */
+    LN_ERR_FLAGS = 8       /* ln_backward_ex: unknown bits in flags */
 } ln_status;
 
 /*
@@ -114,6 +116,64 @@ int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
                 const void *inp, const void *weight, const float *mean,
                 const float *rstd, int64_t N, int64_t C, int dtype,
                 ln_stream_t stream);
+
+/*
+ * LayerNorm forward of a residual sum, the step that precedes LayerNorm in a
+ * GPT-2 block: "llm.c: Large Language Model Training in Pure C/CUDA Without
+ * Dependencies" credits its speed to custom fused kernels (feature list, and
+ * the question "Can llm.c achieve competitive training speeds with
+ * PyTorch?").  Here the residual add is fused into the forward, so the sum is
+ * read from registers instead of being written and read back:
+ *   x         = resid + branch, rounded to dtype (each element rounded once,
+ *               to nearest-even)
+ *   resid_out = x
+ *   out, mean, rstd = ln_forward(x)      (the rounded x, so that the saved
+ *                                         residual and the statistics agree)
+ *   resid_out [N*C] dtype, written       the residual stream after the add
+ *   out, mean, rstd                      as in ln_forward
+ *   resid, branch [N*C] dtype, read      the two summands
+ *   weight, bias [C] dtype, read; eps as in ln_forward
+ * resid_out and out must not overlap each other or any input (no in-place
+ * update).  Bytes moved: 4*N*C*size (two reads, two writes) against 5*N*C*size
+ * for a separate add and ln_forward.  Returns LN_OK or an ln_status error.
+ */
+int ln_forward_residual(void *resid_out, void *out, float *mean, float *rstd,
+                        const void *resid, const void *branch, const void *weight,
+                        const void *bias, int64_t N, int64_t C, float eps, int dtype,
+                        ln_stream_t stream);
+
+/* Flags of ln_backward_ex (bitwise or). */
+/* dinp += the gradient: the previous dinp is read and each sum is rounded to
+ * dtype once.  For a residual stream, whose gradient is the sum of the
+ * branches' gradients ("llm.c: Large Language Model Training in Pure C/CUDA
+ * Without Dependencies", question "How does llm.c handle distributed
+ * multi-GPU training?": gradients are accumulated locally before they are
+ * synchronised). */
+#define LN_BWD_ACCUMULATE_DINP 1u
+/* dweight += and dbias += the column sums (fp32), e.g. over micro-batches of
+ * one optimiser step. */
+#define LN_BWD_ACCUMULATE_DPARAMS 2u
+/* mean and rstd are recomputed from inp (with eps, exactly as ln_forward
+ * computes them) instead of being read; the mean and rstd arguments may then
+ * be NULL.  Saves the 8*N bytes of the saved statistics, and lets a caller
+ * drop them (activation recomputation). */
+#define LN_BWD_RECOMPUTE_STATS 4u
+
+/*
+ * ln_backward with variants: flags == 0 is exactly ln_backward (eps is then
+ * unused).  Arguments as in ln_backward, plus
+ *   eps    finite, > 0; read only with LN_BWD_RECOMPUTE_STATS
+ *   flags  a combination of LN_BWD_ACCUMULATE_DINP, LN_BWD_ACCUMULATE_DPARAMS
+ *          and LN_BWD_RECOMPUTE_STATS; other bits give LN_ERR_FLAGS
+ * With LN_BWD_ACCUMULATE_DINP, dinp is read as well as written (it must hold
+ * the previous gradient); with LN_BWD_ACCUMULATE_DPARAMS, dweight and dbias
+ * are read and N == 0 leaves them unchanged.  The column sums keep their
+ * fixed order, so results stay deterministic.
+ */
+int ln_backward_ex(void *dinp, float *dweight, float *dbias, const void *dout,
+                   const void *inp, const void *weight, const float *mean,
+                   const float *rstd, int64_t N, int64_t C, float eps, int dtype,
+                   unsigned int flags, ln_stream_t stream);
 
 /*
  * ln_backward_noalloc: the same computation and arguments as ln_backward, for
@@ -161,7 +221,7 @@ uint64_t ln_launch_count(void);
  * the current device.  Returns LN_OK, LN_ERR_NULL or LN_ERR_CUDA. */
 int ln_device_status(unsigned int *bits, int clear);
 
-/* Library ABI version: 1. */
+/* Library ABI version: 2 (1 plus ln_forward_residual and ln_backward_ex). */
 int ln_version(void);
 
 #ifdef __cplusplus

@@ -103,44 +103,6 @@ __device__ __forceinline__ void warp_sum2(float &a, float &b) {
     }
 }
 
-// Sum over the W warps of one row (W > 1: all threads of the block work on
-// the same row).  `slot` holds W floats; callers alternate slots so that a
-// slot is never rewritten before every thread has read it.
-template <int W>
-__device__ __forceinline__ float row_sum(float v, float *slot, int warp, int lane) {
-    v = warp_sum(v);
-    if constexpr (W == 1) {
-        return v;
-    } else {
-        if (lane == 0) slot[warp] = v;
-        __syncthreads();
-        float tot = 0.f;
-#pragma unroll
-        for (int k = 0; k < W; ++k) tot += slot[k];
-        return tot;
-    }
-}
-
-template <int W>
-__device__ __forceinline__ void row_sum2(float &a, float &b, float *slot, int warp,
-                                         int lane) {
-    warp_sum2(a, b);
-    if constexpr (W > 1) {
-        if (lane == 0) {
-            slot[warp] = a;
-            slot[W + warp] = b;
-        }
-        __syncthreads();
-        a = 0.f;
-        b = 0.f;
-#pragma unroll
-        for (int k = 0; k < W; ++k) {
-            a += slot[k];
-            b += slot[W + k];
-        }
-    }
-}
-
 // Block-wide sums for the scalar kernels (blockDim.x a multiple of 32).
 __device__ __forceinline__ float block_sum(float v, float *slot, int nwarps) {
     v = warp_sum(v);
@@ -272,6 +234,50 @@ __device__ __forceinline__ void smem_pairs(const float *src, f32x2 (&p)[P]) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Kernel variants, chosen at compile time by a MODE template parameter.
+// ---------------------------------------------------------------------------
+// Forward: the row is x = inp + branch, rounded to T; x is written to
+// resid_out and normalised (the rounded x, so that the saved residual stream
+// and the statistics describe the same values).
+constexpr int kFwdResidual = 1;
+// Backward: dinp += the gradient (the previous dinp is read and the sum is
+// rounded to T once).
+constexpr int kBwdAccumulate = 1;
+// Backward: mean and rstd are recomputed from inp with the forward's
+// pivot-shifted two-pass statistics instead of being read from the arrays.
+constexpr int kBwdRecompute = 2;
+
+// a + b elementwise for two 16-byte vectors of T, each sum rounded to T
+// (fp32: the sum itself; bf16: the fp32 sum is exact or rounds far from a
+// bf16 rounding boundary, so rounding it to nearest-even gives the correctly
+// rounded bf16 sum).
+__device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b, float) {
+    f32x2 pa[2], pb[2];
+    to_pairs(a, pa);
+    to_pairs(b, pb);
+    pa[0] = add2(pa[0], pb[0]);
+    pa[1] = add2(pa[1], pb[1]);
+    return from_pairs(pa);
+}
+__device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b, bf16) {
+    f32x2 pa[4], pb[4];
+    to_pairs(a, pa);
+    to_pairs(b, pb);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) pa[q] = add2(pa[q], pb[q]);
+    return from_pairs(pa);
+}
+template <typename T>
+__device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b) {
+    return add_round(a, b, T());
+}
+// One element of the rounded sum (same value as the vector form).
+template <typename T>
+__device__ __forceinline__ float add_round1(T a, T b) {
+    return to_f32(from_f32<T>(to_f32(a) + to_f32(b)));
+}
+
 // Barrier over the TPR threads of one row group (barrier 0 is the block's;
 // groups use 1 .. GROUPS).
 template <int TPR, int GROUPS>
@@ -344,15 +350,19 @@ __host__ __device__ constexpr size_t bwd_vec_smem(int C) {
 // GROUPS groups.  Rows go round-robin over a persistent grid.  The row is
 // loaded once, turned into deviations from the pivot x[r, 0] and kept in
 // registers as fp32 pairs through both reductions.
-// Requirements (checked by the host): inp, out, weight, bias 16-byte aligned,
-// C * sizeof(T) a multiple of 16, C / E <= V * TPR.
+// With MODE & kFwdResidual the row is inp + branch (rounded to T), which is
+// also written to resid_out.
+// Requirements (checked by the host): inp, out, weight, bias (and branch,
+// resid_out) 16-byte aligned, C * sizeof(T) a multiple of 16, C / E <= V * TPR.
 // ---------------------------------------------------------------------------
-template <typename T, int V, int W, int GROUPS>
+template <typename T, int V, int W, int GROUPS, int MODE = 0>
 __global__ void __launch_bounds__(32 * W * GROUPS)
 ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                   const T *__restrict__ inp, const T *__restrict__ weight,
-                  const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps) {
+                  const T *__restrict__ bias, T *__restrict__ resid_out,
+                  const T *__restrict__ branch, int64_t N, int C, float inv_C, float eps) {
     pdl_enter();
+    constexpr bool RES = (MODE & kFwdResidual) != 0;
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
@@ -381,6 +391,22 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
             const int j = t + i * TPR;
             xv[i] = (j < nvec) ? __ldcs(xr + j) : make_uint4(0u, 0u, 0u, 0u);
         }
+        if constexpr (RES) {
+            const uint4 *br = reinterpret_cast<const uint4 *>(branch) + r * nvec;
+            uint4 *xo = reinterpret_cast<uint4 *>(resid_out) + r * nvec;
+            uint4 bv[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = t + i * TPR;
+                bv[i] = (j < nvec) ? __ldcs(br + j) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int j = t + i * TPR;
+                xv[i] = add_round<T>(xv[i], bv[i]);
+                if (j < nvec) __stcs(xo + j, xv[i]);
+            }
+        }
         float pivot;
         if constexpr (W == 1) {
             float lo, hi;
@@ -388,6 +414,8 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
             to_pairs(xv[0], p0);            // lane 0 holds columns 0 .. E-1
             split(p0[0], lo, hi);
             pivot = __shfl_sync(0xffffffffu, lo, 0);
+        } else if constexpr (RES) {
+            pivot = add_round1<T>(inp[r * C], branch[r * C]);
         } else {
             pivot = to_f32(inp[r * C]);
         }
@@ -452,15 +480,21 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
 // and partial[b][C:2C] (dbias part).
 //   dinp = rstd * (g - mean(g) - xhat * mean(g xhat)) is evaluated as
 //   fma(g, rstd, fma(xhat, -rstd*mean(g xhat), -rstd*mean(g))).
+// MODE & kBwdAccumulate: the previous dinp vector is loaded where the new one
+// is formed and added before rounding.  MODE & kBwdRecompute: mean and rstd come from the
+// row itself (pivot x[r, 0], deviations d = (x - pivot) - mean(x - pivot),
+// rstd = 1/sqrt(mean(d^2) + eps)), and xhat = d * rstd.
 // ---------------------------------------------------------------------------
-template <typename T, int V, int W, int GROUPS>
+template <typename T, int V, int W, int GROUPS, int MODE = 0>
 __global__ void __launch_bounds__(32 * W * GROUPS, 32 * W * GROUPS <= 256 ? 2 : 1)
 ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ dout, const T *__restrict__ inp,
                   const T *__restrict__ weight, const float *__restrict__ mean,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
-                  int64_t rows_per_block) {
+                  int64_t rows_per_block, float eps) {
     pdl_enter();
+    constexpr bool ACC = (MODE & kBwdAccumulate) != 0;
+    constexpr bool RECOMP = (MODE & kBwdRecompute) != 0;
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
@@ -495,6 +529,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     for (int64_t r = row0 + group; r < row1; r += GROUPS) {
         const uint4 *xr = reinterpret_cast<const uint4 *>(inp) + r * nvec;
         const uint4 *dr = reinterpret_cast<const uint4 *>(dout) + r * nvec;
+        uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
         uint4 xv[V], dv[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
@@ -507,10 +542,63 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 dv[i] = xv[i];
             }
         }
-        const float m = __ldg(mean + r);
-        const float s = __ldg(rstd + r);
-        const f32x2 M = pair(m, m);
+        // xhat = (x - K) * S, or ((x - K) - MD) * S when recomputing
+        float s;
+        f32x2 K, MD = pair(0.f, 0.f);
+        if constexpr (RECOMP) {
+            float pivot;
+            if constexpr (W == 1) {
+                float lo, hi;
+                f32x2 p0[P];
+                to_pairs(xv[0], p0);        // lane 0 holds columns 0 .. E-1
+                split(p0[0], lo, hi);
+                pivot = __shfl_sync(0xffffffffu, lo, 0);
+            } else {
+                pivot = to_f32(inp[r * C]);
+            }
+            K = pair(pivot, pivot);
+            f32x2 sd = pair(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                if (t + i * TPR < nvec) {
+                    f32x2 x[P];
+                    to_pairs(xv[i], x);
+#pragma unroll
+                    for (int k = 0; k < P; ++k) sd = add2(sd, sub2(x[k], K));
+                }
+            }
+            const float md =
+                group_sum<W, GROUPS>(hsum(sd), s_red + parity * 2 * W, group, warp, lane) * inv_C;
+            parity ^= 1;
+            MD = pair(md, md);
+            f32x2 sq = pair(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                if (t + i * TPR < nvec) {
+                    f32x2 x[P];
+                    to_pairs(xv[i], x);
+#pragma unroll
+                    for (int k = 0; k < P; ++k) {
+                        const f32x2 d = sub2(sub2(x[k], K), MD);
+                        sq = fma2(d, d, sq);
+                    }
+                }
+            }
+            const float var =
+                group_sum<W, GROUPS>(hsum(sq), s_red + parity * 2 * W, group, warp, lane) * inv_C;
+            parity ^= 1;
+            s = rsqrtf(var + eps);
+        } else {
+            const float m = __ldg(mean + r);
+            s = __ldg(rstd + r);
+            K = pair(m, m);
+        }
         const f32x2 S = pair(s, s);
+        auto xhat = [&](f32x2 x) {
+            f32x2 d = sub2(x, K);
+            if constexpr (RECOMP) d = sub2(d, MD);
+            return mul2(d, S);
+        };
 
         f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
 #pragma unroll
@@ -523,7 +611,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
                 for (int k = 0; k < P; ++k) {
-                    const f32x2 xh = mul2(sub2(x[k], M), S);
+                    const f32x2 xh = xhat(x[k]);
                     const f32x2 g = mul2(dy[k], wp[k]);
                     s1 = add2(s1, g);
                     s2 = fma2(g, xh, s2);
@@ -538,7 +626,6 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
         const f32x2 NA = pair(na, na);
         const f32x2 NC = pair(nc, nc);
 
-        uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + i * TPR;
@@ -549,11 +636,17 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
                 for (int k = 0; k < P; ++k) {
-                    const f32x2 xh = mul2(sub2(x[k], M), S);
+                    const f32x2 xh = xhat(x[k]);
                     const f32x2 g = mul2(dy[k], wp[k]);
                     o[k] = fma2(g, S, fma2(xh, NC, NA));
                     acc_w[i][k] = fma2(dy[k], xh, acc_w[i][k]);
                     acc_b[i][k] = add2(acc_b[i][k], dy[k]);
+                }
+                if constexpr (ACC) {
+                    f32x2 pp[P];
+                    to_pairs(__ldcs(gr + j), pp);
+#pragma unroll
+                    for (int k = 0; k < P; ++k) o[k] = add2(o[k], pp[k]);
                 }
                 __stcs(gr + j, from_pairs(o));
             }
@@ -626,13 +719,14 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
 // of the 2C flattened columns with S = kColsumThreads/32 slices: slice y sums
 // the partial rows b = y, y + S, ... in increasing order (16 loads issued
 // before their adds), then slice 0 adds the S slice sums in order.  The order
-// depends on G only, so the result is deterministic.
+// depends on G only, so the result is deterministic.  With accumulate != 0
+// the previous dweight[c] / dbias[c] is added to the finished sum.
 // ---------------------------------------------------------------------------
 constexpr int kColsumThreads = 1024;
 
 static __global__ void __launch_bounds__(kColsumThreads)
 ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
-                 const float *__restrict__ partial, int G, int C) {
+                 const float *__restrict__ partial, int G, int C, int accumulate) {
     pdl_enter();
     constexpr int S = kColsumThreads / 32;
     __shared__ float s[S][33];
@@ -659,10 +753,9 @@ ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
         float tot = s[0][tx];
 #pragma unroll
         for (int k = 1; k < S; ++k) tot += s[k][tx];
-        if (j < C)
-            dweight[j] = tot;
-        else
-            dbias[j - C] = tot;
+        float *dst = j < C ? dweight + j : dbias + (j - C);
+        if (accumulate) tot = *dst + tot;
+        *dst = tot;
     }
 }
 
@@ -671,13 +764,15 @@ ln_colsum_kernel(float *__restrict__ dweight, float *__restrict__ dbias,
 // scalar load (coalesced across the threads of a row); the row is re-read
 // from L1/L2 for each pass instead of being held in registers.
 // ---------------------------------------------------------------------------
-template <typename T, bool BLOCK_ROW>
+template <typename T, bool BLOCK_ROW, int MODE = 0>
 __global__ void __launch_bounds__(512)
 ln_fwd_scalar_kernel(T *__restrict__ out, float *__restrict__ mean,
                      float *__restrict__ rstd, const T *__restrict__ inp,
-                     const T *__restrict__ weight, const T *__restrict__ bias, int64_t N,
+                     const T *__restrict__ weight, const T *__restrict__ bias,
+                     T *__restrict__ resid_out, const T *__restrict__ branch, int64_t N,
                      int C, float inv_C, float eps) {
     pdl_enter();
+    constexpr bool RES = (MODE & kFwdResidual) != 0;
     __shared__ float s_red[2][32];
     const int tpr = BLOCK_ROW ? (int)blockDim.x : 32;
     const int groups = blockDim.x / tpr;
@@ -688,22 +783,33 @@ ln_fwd_scalar_kernel(T *__restrict__ out, float *__restrict__ mean,
     for (int64_t r = (int64_t)blockIdx.x * groups + group; r < N;
          r += (int64_t)gridDim.x * groups) {
         const T *x = inp + r * C;
-        const float pivot = to_f32(x[0]);
+        const T *br = branch + (RES ? r * C : 0);
+        // element c of the row (the rounded sum in the residual variant)
+        auto xc = [&](int c) {
+            if constexpr (RES)
+                return add_round1<T>(x[c], br[c]);
+            else
+                return to_f32(x[c]);
+        };
+        const float pivot = xc(0);
         float s = 0.f;
-        for (int c = t; c < C; c += tpr) s += to_f32(x[c]) - pivot;
+        for (int c = t; c < C; c += tpr) s += xc(c) - pivot;
         s = block_sum(s, s_red[0], nwarps);
         const float mean_d = s * inv_C;
         float q = 0.f;
         for (int c = t; c < C; c += tpr) {
-            const float d = (to_f32(x[c]) - pivot) - mean_d;
+            const float d = (xc(c) - pivot) - mean_d;
             q += d * d;
         }
         q = block_sum(q, s_red[1], nwarps);
         const float rs = rsqrtf(q * inv_C + eps);
         T *y = out + r * C;
-        for (int c = t; c < C; c += tpr)
-            y[c] = from_f32<T>(((to_f32(x[c]) - pivot) - mean_d) * rs * to_f32(weight[c]) +
+        for (int c = t; c < C; c += tpr) {
+            const float v = xc(c);
+            if constexpr (RES) resid_out[r * C + c] = from_f32<T>(v);
+            y[c] = from_f32<T>(((v - pivot) - mean_d) * rs * to_f32(weight[c]) +
                                to_f32(bias[c]));
+        }
         if (t == 0) {
             mean[r] = pivot + mean_d;
             rstd[r] = rs;
@@ -715,14 +821,16 @@ ln_fwd_scalar_kernel(T *__restrict__ out, float *__restrict__ mean,
 // and accumulates its column sums directly in the block's partial row
 // (written on the block's first row, added to afterwards; zero-filled when
 // the block has no rows).
-template <typename T>
+template <typename T, int MODE = 0>
 __global__ void __launch_bounds__(512)
 ln_bwd_scalar_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                      const T *__restrict__ dout, const T *__restrict__ inp,
                      const T *__restrict__ weight, const float *__restrict__ mean,
                      const float *__restrict__ rstd, int64_t N, int C, float inv_C,
-                     int64_t rows_per_block) {
+                     int64_t rows_per_block, float eps) {
     pdl_enter();
+    constexpr bool ACC = (MODE & kBwdAccumulate) != 0;
+    constexpr bool RECOMP = (MODE & kBwdRecompute) != 0;
     __shared__ float s_red[2][64];
     const int tpr = blockDim.x;
     const int nwarps = tpr >> 5;
@@ -735,11 +843,31 @@ ln_bwd_scalar_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     for (int64_t r = row0; r < row1; ++r) {
         const T *x = inp + r * C;
         const T *dy = dout + r * C;
-        const float m = mean[r];
-        const float s = rstd[r];
+        // xhat = ((x - K) - md) * s: K = mean[r], md = 0 from the saved
+        // statistics, or the pivot x[r, 0] and the mean deviation from it
+        float K, md = 0.f, s;
+        if constexpr (RECOMP) {
+            K = to_f32(x[0]);
+            float sd = 0.f;
+            for (int c = threadIdx.x; c < C; c += tpr) sd += to_f32(x[c]) - K;
+            sd = block_sum(sd, s_red[parity], nwarps);
+            parity ^= 1;
+            md = sd * inv_C;
+            float q = 0.f;
+            for (int c = threadIdx.x; c < C; c += tpr) {
+                const float d = (to_f32(x[c]) - K) - md;
+                q += d * d;
+            }
+            q = block_sum(q, s_red[parity], nwarps);
+            parity ^= 1;
+            s = rsqrtf(q * inv_C + eps);
+        } else {
+            K = mean[r];
+            s = rstd[r];
+        }
         float s1 = 0.f, s2 = 0.f;
         for (int c = threadIdx.x; c < C; c += tpr) {
-            const float xh = (to_f32(x[c]) - m) * s;
+            const float xh = ((to_f32(x[c]) - K) - md) * s;
             const float g = to_f32(dy[c]) * to_f32(weight[c]);
             s1 += g;
             s2 += g * xh;
@@ -751,9 +879,11 @@ ln_bwd_scalar_kernel(T *__restrict__ dinp, float *__restrict__ partial,
         T *gx = dinp + r * C;
         for (int c = threadIdx.x; c < C; c += tpr) {
             const float dyc = to_f32(dy[c]);
-            const float xh = (to_f32(x[c]) - m) * s;
+            const float xh = ((to_f32(x[c]) - K) - md) * s;
             const float g = dyc * to_f32(weight[c]);
-            gx[c] = from_f32<T>(s * (g - a - xh * cc));
+            float v = s * (g - a - xh * cc);
+            if constexpr (ACC) v += to_f32(gx[c]);
+            gx[c] = from_f32<T>(v);
             if (first) {
                 pw[c] = dyc * xh;
                 pb[c] = dyc;

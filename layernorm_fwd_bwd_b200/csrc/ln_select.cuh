@@ -1,14 +1,17 @@
-// ln_select.cuh -- which vectorised kernel variant serves a row of nvec
-// 16-byte vectors.  Shared by every launcher so that the variant and its
-// shared-memory size are chosen in exactly one place.
+// ln_select.cuh -- which kernel variant serves a row of nvec 16-byte vectors.
+// Shared by every launcher so that the variant and its shared-memory size are
+// chosen in exactly one place.
 //
-// Forward: one warp per row (8 rows per 256-thread block) while the row fits
-// in V <= 8 vectors per lane; wider rows use W = 4, 8 or 16 warps per row with
-// 4 vectors per thread.  Backward: the per-thread column accumulators
-// (2 * V * E floats) stay at or below 64 registers, so one warp per row serves
-// up to V = 6 (fp32) / 4 (bf16) vectors per lane and wider rows use W = 2, 4,
-// 8 or 16 warps per row with 4 vectors per thread.  Blocks hold 256 threads
-// (512 for W = 16).  Rows wider than the widest variant take the scalar path.
+// Forward: rows of up to 8 vectors per lane take the one-shot tile kernel
+// (ln_tile.cuh): one warp per row up to 4 vectors, two warps per row for 5..8;
+// wider rows take the persistent register-resident kernel with W = 4, 8 or 16
+// warps per row and 4 vectors per thread.
+// Backward: rows of up to 4 (bf16) / 6 (fp32) vectors per lane take the
+// persistent TMA-ring kernel (ln_tma.cuh) on one warp per row, wider rows the
+// ring with W = 2..4 warps per row; rows wider than that take the
+// register-resident kernel (W = 4..16 warps per row, 4 vectors per thread).
+// Rows wider than the widest variant, and any misaligned call, take the
+// scalar kernels.
 #pragma once
 
 #include "ln_kernels.cuh"
@@ -21,42 +24,22 @@
 #ifndef LN_BWD_GROUPS_W1
 #define LN_BWD_GROUPS_W1 8
 #endif
-
-// Rows served by one warp each: the forward runs, by default, the one-shot
-// tile kernel (ln_tile.cuh; style 2) and the backward the persistent TMA-ring
-// kernel (ln_tma.cuh; style 1).  Style 0 selects the persistent
-// register-resident kernels (ln_kernels.cuh).  Measured on B200 at GPT-2 124M
-// shapes: forward tile 35 us vs ring 45 us vs register 41 us; backward ring
-// 59 us vs register 65 us vs cluster tile 120 us.
-#ifndef LN_FWD_STYLE
-#define LN_FWD_STYLE 2
-#endif
-#ifndef LN_BWD_STYLE
-#define LN_BWD_STYLE 1
-#endif
 #ifndef LN_BWD_RING_RR
 #define LN_BWD_RING_RR 1          // ring backward: tiles round-robin over blocks
 #endif
 #ifndef LN_TILE_FWD_TILES
 #define LN_TILE_FWD_TILES 2       // tiles of 8 rows per forward block
 #endif
-#ifndef LN_TILE_BWD_TILES
-#define LN_TILE_BWD_TILES 2       // tiles of 8 rows per backward block
-#endif
-#ifndef LN_TILE_CLUSTER
-#define LN_TILE_CLUSTER 8         // backward blocks per cluster
-#endif
 
 namespace lnk {
 
+// Largest dynamic shared memory of one block on sm_100 (227 KB).
+constexpr size_t kMaxSmemPerBlock = 232448;
+
 // consumer warps (= rows per tile) per block; the producer warp comes on top
-#ifndef LN_TMA_FWD_CONSUMERS
-#define LN_TMA_FWD_CONSUMERS 8
-#endif
 #ifndef LN_TMA_BWD_CONSUMERS
 #define LN_TMA_BWD_CONSUMERS 15   // + 1 producer warp: 512 threads, one block per SM
 #endif
-constexpr int kTmaFwdConsumers = LN_TMA_FWD_CONSUMERS;
 constexpr int kTmaBwdConsumers = LN_TMA_BWD_CONSUMERS;
 // consumer warps of the backward ring when W warps share a row
 template <int W> struct BwdRingConsumers {
@@ -70,31 +53,37 @@ template <int W> struct BwdRingConsumers {
 #endif
 constexpr int kTileWarps = 8;                 // warps (= rows per tile) per tile block
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
-constexpr int kTileBwdTiles = LN_TILE_BWD_TILES;
-constexpr int kTileCluster = LN_TILE_CLUSTER;
 
-// Ring depth: a stage holds 7-8 rows of up to 32*V 16-byte vectors (twice
-// that in the backward, inp and dout); keep the ring near 48-96 KB per block.
-template <int V> struct FwdStages { static constexpr int value = V <= 4 ? 4 : 2; };
+// Arrays streamed through the backward ring: inp and dout, plus the previous
+// dinp when accumulating.
+template <int MODE> struct BwdRingArrays {
+    static constexpr int value = (MODE & kBwdAccumulate) ? 3 : 2;
+};
+
 #ifndef LN_TMA_BWD_STAGES
 #define LN_TMA_BWD_STAGES 0       // 0: from the shared-memory budget (below)
 #endif
-// Backward ring depth: as many stages (2..6) of NC rows of inp and dout, at
-// up to 32*V*16 bytes a row, as fit in about 200 KB for one block per SM
-// (100 KB at two).  Measured: a deeper ring lifts fp32 rows from 5.6 to
-// 6.2 TB/s.
-template <int V, int NC> struct BwdStages {
-    static constexpr size_t kBudget = (NC + 1) * 32 <= 256 ? (100u << 10) : (200u << 10);
-    static constexpr size_t kStage = size_t(NC) * 2 * 32 * V * 16;
+// Backward ring depth: as many stages (2..6) of NC rows of NS arrays, at up to
+// 32*V*16 bytes a row, as fit in about 200 KB (208 KB with three arrays) for
+// one block per SM (100 KB at two).  Measured: a deeper ring lifts fp32 rows
+// from 5.6 to 6.2 TB/s.
+template <int V, int NC, int NS = 2> struct BwdStages {
+    static constexpr size_t kBudget = (NC + 1) * 32 <= 256 ? (100u << 10)
+                                      : NS > 2             ? (208u << 10)
+                                                           : (200u << 10);
+    static constexpr size_t kStage = size_t(NC) * NS * 32 * V * 16;
     static constexpr int kFit = int(kBudget / kStage);
     static constexpr int value =
         LN_TMA_BWD_STAGES ? LN_TMA_BWD_STAGES : (kFit < 2 ? 2 : (kFit > 6 ? 6 : kFit));
 };
 
-// Backward, one warp per row: at most 6 (fp32) / 4 (bf16) vectors per lane,
-// i.e. at most 48 / 64 column accumulators per thread.
-template <typename T> struct BwdVmaxW1 { static constexpr int value = 6; };
-template <> struct BwdVmaxW1<bf16> { static constexpr int value = 4; };
+// Shared memory of a ring variant at the widest row it serves.
+template <typename T, int V, int W, int NS>
+constexpr size_t bwd_ring_smem_max() {
+    constexpr int NC = BwdRingConsumers<W>::value;
+    constexpr int S = BwdStages<V, NC, NS>::value;
+    return bwd_tma_smem<T, NC, S, W, NS>(32 * W * V * Vec<T>::E);
+}
 
 // Calls visitor.template run<V, W, GROUPS>() for the forward variant; returns
 // false when no vectorised variant covers nvec.
@@ -118,27 +107,45 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
 }
 
 // Backward ring (ln_tma.cuh).  One warp per row while a lane holds at most
-// 4 (bf16) / 6 (fp32) vectors; wider rows are split over W = 2..4 warps with
-// 3 (bf16) / 5 (fp32) vectors per lane, which keeps x - mean in registers
-// between the two passes.  Measured on B200: bf16 C = 1024 is faster on one
-// warp (4 vectors, recomputing x - mean) than on two (the row-group exchange
-// costs more than it saves); C = 1600 is faster on three warps (43 us) than
-// on two with 4 vectors (46 us).  Calls visitor.template ring<V, W>();
-// false when rows are wider than 4 warps cover.
-template <typename T> struct RingVmax { static constexpr int one = 6, shared = 5; };
-template <> struct RingVmax<bf16> { static constexpr int one = 4, shared = 3; };
+// `one` vectors; wider rows are split over W = 2..4 warps with `shared`
+// vectors per lane, which keeps x - mean in registers between the two
+// passes.  Measured on B200: bf16 C = 1024 is faster on one warp (4 vectors,
+// recomputing x - mean) than on two (the row-group exchange costs more than
+// it saves); C = 1600 is faster on three warps (43 us) than on two with 4
+// vectors (46 us).  With three arrays per stage (accumulating) a stage is
+// half as large again, so fp32 rows stop at 4 vectors per lane, where two
+// stages of the widest rows still fit in shared memory; recomputing the
+// statistics, bf16 rows of 4 vectors per lane would spill, so they go to two
+// warps.
+template <typename T, int MODE> struct RingVmax;
+template <int MODE> struct RingVmax<float, MODE> {
+    static constexpr bool kAcc = (MODE & kBwdAccumulate) != 0;
+    static constexpr int one = kAcc ? 4 : 6, shared = kAcc ? 4 : 5;
+};
+template <int MODE> struct RingVmax<bf16, MODE> {
+    static constexpr int one = (MODE & kBwdRecompute) ? 3 : 4, shared = 3;
+};
 
-template <typename T, typename Visitor>
+// Calls visitor.template ring<V, W>(); false when rows are wider than 4 warps
+// cover.
+template <typename T, int MODE, typename Visitor>
 bool visit_bwd_ring(int nvec, Visitor &v) {
-    constexpr int V1 = RingVmax<T>::one;
-    constexpr int VS = RingVmax<T>::shared;
+    constexpr int NS = BwdRingArrays<MODE>::value;
+    constexpr int V1 = RingVmax<T, MODE>::one;
+    constexpr int VS = RingVmax<T, MODE>::shared;
+    static_assert(bwd_ring_smem_max<T, V1, 1, NS>() <= kMaxSmemPerBlock, "ring fits");
+    static_assert(bwd_ring_smem_max<T, VS, 2, NS>() <= kMaxSmemPerBlock, "ring fits");
+    static_assert(bwd_ring_smem_max<T, VS, 3, NS>() <= kMaxSmemPerBlock, "ring fits");
+    static_assert(bwd_ring_smem_max<T, VS, 4, NS>() <= kMaxSmemPerBlock, "ring fits");
     const int v1 = (nvec + 31) / 32;
     switch (v1) {
         case 1: v.template ring<1, 1>(); return true;
         case 2: v.template ring<2, 1>(); return true;
         case 3: v.template ring<3, 1>(); return true;
-        case 4: v.template ring<4, 1>(); return true;
         default: break;
+    }
+    if constexpr (V1 >= 4) {
+        if (v1 == 4) { v.template ring<4, 1>(); return true; }
     }
     if constexpr (V1 > 4) {
         if (v1 == 5) { v.template ring<5, 1>(); return true; }
@@ -153,27 +160,12 @@ bool visit_bwd_ring(int nvec, Visitor &v) {
     }
 }
 
+// Backward rows wider than the ring covers (more than 4 * 32 * shared
+// vectors): the register-resident kernel with W = 4, 8 or 16 warps per row
+// and 4 vectors per thread.  Calls visitor.template run<V, W, GROUPS>();
+// false when rows are wider still.
 template <typename T, typename Visitor>
 bool visit_bwd_vec(int nvec, Visitor &v) {
-    constexpr int VM = BwdVmaxW1<T>::value;
-    const int v1 = (nvec + 31) / 32;
-    if (v1 <= VM) {
-        switch (v1) {
-            case 1: v.template run<1, 1, LN_BWD_GROUPS_W1>(); return true;
-            case 2: v.template run<2, 1, LN_BWD_GROUPS_W1>(); return true;
-            case 3: v.template run<3, 1, LN_BWD_GROUPS_W1>(); return true;
-            case 4: v.template run<4, 1, LN_BWD_GROUPS_W1>(); return true;
-            default: break;
-        }
-        if constexpr (VM > 4) {
-            switch (v1) {
-                case 5: v.template run<5, 1, LN_BWD_GROUPS_W1>(); return true;
-                case 6: v.template run<6, 1, LN_BWD_GROUPS_W1>(); return true;
-                default: break;
-            }
-        }
-    }
-    if (nvec <= 2 * 32 * 4) { v.template run<4, 2, 4>(); return true; }
     if (nvec <= 4 * 32 * 4) { v.template run<4, 4, 2>(); return true; }
     if (nvec <= 8 * 32 * 4) { v.template run<4, 8, 1>(); return true; }
     if (nvec <= 16 * 32 * 4) { v.template run<4, 16, 1>(); return true; }

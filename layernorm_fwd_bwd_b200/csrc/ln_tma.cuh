@@ -98,35 +98,33 @@ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? 
 
 // Shared memory layout (bytes):
 //   [0, 128)            full[S], empty[S] mbarriers (S <= 8)
-//   [128, 128 + A)      fp32 parameters: weight (+ bias in the forward), A = n*C*4 rounded up
-//   [.., + S * stage)   the ring; stage = rows * row_bytes * (1 fwd, 2 bwd)
+//   [128, 128 + A)      weight as fp32, A = C*4 rounded up to 128
+//   [.., + S * stage)   the ring; stage = NS arrays (inp, dout and, when
+//                       accumulating, the previous dinp) of the tile's rows
+//   [.., ..)            row-group exchange slots (W > 1)
 template <typename T>
-__host__ __device__ constexpr size_t tma_ring_offset(int C, int nparams) {
-    return 128 + align128(size_t(nparams) * C * 4);
+__host__ __device__ constexpr size_t tma_ring_offset(int C) {
+    return 128 + align128(size_t(C) * 4);
 }
-template <typename T, int NC, int S>
-__host__ __device__ constexpr size_t fwd_tma_smem(int C) {
-    return tma_ring_offset<T>(C, 2) + size_t(S) * NC * C * sizeof(T);
-}
-template <typename T, int NC, int S, int W>
+template <typename T, int NC, int S, int W, int NS>
 __host__ __device__ constexpr size_t bwd_tma_ring_bytes(int C) {
-    // the ring (NC/W rows of inp and dout per stage), also reused for the
+    // the ring (NC/W rows of each array per stage), also reused for the
     // end-of-block combine: at most half the row groups (rounded up) park
     // 2C floats each
-    const size_t ring = size_t(S) * (NC / W) * 2 * C * sizeof(T);
+    const size_t ring = size_t(S) * (NC / W) * NS * C * sizeof(T);
     const size_t comb = size_t((NC / W + 1) / 2) * 2 * C * 4;
     return ring > comb ? ring : comb;
 }
-template <typename T, int NC, int S, int W = 1>
+template <typename T, int NC, int S, int W, int NS>
 __host__ __device__ constexpr size_t bwd_tma_smem(int C) {
     // weight as fp32 (read twice per row: unpacking bf16 there costs more
     // issue slots than the wider shared-memory reads), the ring, and the
     // row-group exchange slots when rows are shared by W > 1 warps
-    return tma_ring_offset<T>(C, 1) + align128(bwd_tma_ring_bytes<T, NC, S, W>(C)) +
+    return tma_ring_offset<T>(C) + align128(bwd_tma_ring_bytes<T, NC, S, W, NS>(C)) +
            (W > 1 ? size_t(NC / W) * 2 * 3 * W * 4 : 0);
 }
 
-// Producer side, shared by both kernels: stream tiles k = 0, 1, ... of this
+// Producer side: stream tiles k = 0, 1, ... of this
 // block (tile index tile_of(k)) into the ring.  Before returning -- after the
 // last tile, or after recording an error -- it waits (bounded) until its
 // last copies have landed, so the block never exits with a copy still
@@ -147,144 +145,6 @@ __device__ __forceinline__ void tma_produce(uint64_t *full, uint64_t *empty,
     }
     for (int64_t q = (k > S ? k - S : 0); q < k; ++q)
         if (!mbar_wait(&full[q % S], uint32_t((q / S) & 1))) atomicOr(status, kStatusDrain);
-}
-
-// ---------------------------------------------------------------------------
-// Forward.  Tile = NC consecutive rows (NC consumer warps, one row each);
-// tiles go round-robin over a persistent grid.  Warp NC is the producer.
-// Requirements (checked by the host): inp/out/weight/bias 16-byte aligned,
-// C * sizeof(T) a multiple of 16, C / E <= 32 * V.
-// ---------------------------------------------------------------------------
-template <typename T, int V, int NC, int S>
-__global__ void __launch_bounds__(32 * (NC + 1))
-ln_fwd_tma_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
-                  const T *__restrict__ inp, const T *__restrict__ weight,
-                  const T *__restrict__ bias, int64_t N, int C, float inv_C, float eps,
-                  unsigned *__restrict__ status) {
-    pdl_enter();
-    static_assert(S >= 2 && S <= 8, "ring depth");
-    constexpr int E = Vec<T>::E;
-    constexpr int P = E / 2;
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + S;
-    float *s_w = reinterpret_cast<float *>(smem + 128);
-    float *s_b = s_w + C;
-    unsigned char *ring = smem + tma_ring_offset<T>(C, 2);
-    const int nvec = C / E;
-    const uint32_t row_bytes = uint32_t(C) * sizeof(T);
-    const uint32_t stage_bytes = NC * row_bytes;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NC);
-        }
-        fence_mbar_init();
-    }
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-        s_w[c] = to_f32(weight[c]);
-        s_b[c] = to_f32(bias[c]);
-    }
-    __syncthreads();
-
-    const int64_t ntiles = (N + NC - 1) / NC;
-    const int64_t ntiles_here =
-        blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-
-    if (warp == NC) {
-        if (lane == 0) {
-            tma_produce<S>(
-                full, empty, ntiles_here, status,
-                [&](int64_t k) { return int64_t(blockIdx.x) + k * gridDim.x; },
-                [&](int64_t tile, int st, uint64_t *bar) {
-                    const int64_t row0 = tile * NC;
-                    const uint32_t bytes = uint32_t(min64(NC, N - row0)) * row_bytes;
-                    mbar_arrive_expect_tx(bar, bytes);
-                    bulk_load(ring + size_t(st) * stage_bytes,
-                              reinterpret_cast<const unsigned char *>(inp) + row0 * row_bytes,
-                              bytes, bar);
-                });
-        }
-        return;
-    }
-
-    for (int64_t k = 0; k < ntiles_here; ++k) {
-        const int st = int(k % S);
-        if (!mbar_wait(&full[st], uint32_t((k / S) & 1))) {
-            if (lane == 0) atomicOr(status, kStatusWaitFull);
-            break;
-        }
-        const int64_t r = (int64_t(blockIdx.x) + k * gridDim.x) * NC + warp;
-        const bool valid = r < N;                   // warp-uniform
-        const uint4 *src =
-            reinterpret_cast<const uint4 *>(ring + size_t(st) * stage_bytes + warp * row_bytes);
-        uint4 xv[V];
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int j = lane + 32 * i;
-            xv[i] = (valid && j < nvec) ? src[j] : make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();                   // reads done before the refill
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);     // stage slot read: release it
-        if (!valid) continue;
-
-        float pivot;
-        {
-            float lo, hi;
-            f32x2 p0[P];
-            to_pairs(xv[0], p0);
-            split(p0[0], lo, hi);
-            pivot = __shfl_sync(0xffffffffu, lo, 0);
-        }
-        const f32x2 K = pair(pivot, pivot);
-        f32x2 d[V][P];
-        f32x2 acc = pair(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const bool ok = lane + 32 * i < nvec;
-            to_pairs(xv[i], d[i]);
-#pragma unroll
-            for (int q = 0; q < P; ++q) {
-                d[i][q] = sub2(d[i][q], K);
-                if (ok) acc = add2(acc, d[i][q]);
-            }
-        }
-        const float mean_d = warp_sum(hsum(acc)) * inv_C;
-        const f32x2 M = pair(mean_d, mean_d);
-        f32x2 sq = pair(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const bool ok = lane + 32 * i < nvec;
-#pragma unroll
-            for (int q = 0; q < P; ++q) {
-                d[i][q] = sub2(d[i][q], M);
-                if (ok) sq = fma2(d[i][q], d[i][q], sq);
-            }
-        }
-        const float rs = rsqrtf(warp_sum(hsum(sq)) * inv_C + eps);
-        const f32x2 R = pair(rs, rs);
-        uint4 *yr = reinterpret_cast<uint4 *>(out) + r * nvec;
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int j = lane + 32 * i;
-            if (j < nvec) {
-                f32x2 wp[P], bp[P], o[P];
-                smem_pairs<P>(s_w + j * E, wp);
-                smem_pairs<P>(s_b + j * E, bp);
-#pragma unroll
-                for (int q = 0; q < P; ++q) o[q] = fma2(mul2(d[i][q], R), wp[q], bp[q]);
-                __stcs(yr + j, from_pairs(o));
-            }
-        }
-        if (lane == 0) {
-            mean[r] = pivot + mean_d;
-            rstd[r] = rs;
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -323,24 +183,30 @@ __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, f
 // 512-thread block, one per SM, 128 registers per thread), W warps per row,
 // so a tile holds RT = NC / W consecutive rows; tiles go round-robin over
 // the persistent grid (RR) or in contiguous ranges.  A stage holds the tile's
-// inp rows followed by its dout rows.  Warp w serves row w / W of each tile
-// and, within it, vectors j = (w % W) * 32 + lane + i * 32 * W; it keeps
+// inp rows, then its dout rows and, when accumulating (MODE &
+// kBwdAccumulate), the previous dinp rows.  Warp w serves row w / W of each
+// tile and, within it, vectors j = (w % W) * 32 + lane + i * 32 * W; it keeps
 // dout*xhat and dout for those columns in registers.  Row sums of the W warps
 // of a row meet in shared memory (group_exchange).  At the end the RT row
 // groups are added in a fixed tree (warps owning the same columns only) and
 // the warps of group 0 write the block's partial row.  mean/rstd of the next
-// row are prefetched one tile ahead.
+// row are prefetched one tile ahead; with MODE & kBwdRecompute they are not
+// read at all but recomputed from the staged row (pivot x[r, 0], two-pass
+// deviations, as in the forward).
 // ---------------------------------------------------------------------------
-template <typename T, int V, int NC, int S, bool RR, int W = 1>
+template <typename T, int V, int NC, int S, bool RR, int W = 1, int MODE = 0>
 __global__ void __launch_bounds__(32 * (NC + 1), (NC + 1) * 32 <= 256 ? 2 : 1)
 ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                   const T *__restrict__ dout, const T *__restrict__ inp,
                   const T *__restrict__ weight, const float *__restrict__ mean,
                   const float *__restrict__ rstd, int64_t N, int C, float inv_C,
-                  int64_t tiles_per_block, unsigned *__restrict__ status) {
+                  int64_t tiles_per_block, float eps, unsigned *__restrict__ status) {
     pdl_enter();
     static_assert(S >= 2 && S <= 8, "ring depth");
     static_assert(NC % W == 0 && NC / W >= 2 && NC / W <= 15, "row groups");
+    constexpr bool ACC = (MODE & kBwdAccumulate) != 0;
+    constexpr bool RECOMP = (MODE & kBwdRecompute) != 0;
+    constexpr int NS = ACC ? 3 : 2;                          // arrays per stage
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int RT = NC / W;                               // rows per tile
@@ -349,13 +215,13 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + S;
     float *s_w = reinterpret_cast<float *>(smem + 128);      // weight as fp32
-    unsigned char *ring = smem + tma_ring_offset<T>(C, 1);
+    unsigned char *ring = smem + tma_ring_offset<T>(C);
     const int nvec = C / E;
     const uint32_t row_bytes = uint32_t(C) * sizeof(T);
-    const uint32_t half_bytes = RT * row_bytes;              // inp part of a stage
-    const uint32_t stage_bytes = 2 * half_bytes;
+    const uint32_t half_bytes = RT * row_bytes;              // one array of a stage
+    const uint32_t stage_bytes = NS * half_bytes;
     float *s_red = reinterpret_cast<float *>(
-        ring + align128(bwd_tma_ring_bytes<T, NC, S, W>(C)));   // [RT][2][3W] (W > 1)
+        ring + align128(bwd_tma_ring_bytes<T, NC, S, W, NS>(C)));   // [RT][2][3W] (W > 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int group = warp / W;                              // row in the tile
@@ -400,20 +266,25 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 [&](int64_t tile, int st, uint64_t *bar) {
                     const int64_t row0 = tile * RT;
                     const uint32_t bytes = uint32_t(min64(RT, N - row0)) * row_bytes;
-                    mbar_arrive_expect_tx(bar, 2 * bytes);
+                    mbar_arrive_expect_tx(bar, NS * bytes);
                     unsigned char *dst = ring + size_t(st) * stage_bytes;
                     bulk_load(dst, reinterpret_cast<const unsigned char *>(inp) + row0 * row_bytes,
                               bytes, bar);
                     bulk_load(dst + half_bytes,
                               reinterpret_cast<const unsigned char *>(dout) + row0 * row_bytes,
                               bytes, bar);
+                    if constexpr (ACC)
+                        bulk_load(dst + 2 * half_bytes,
+                                  reinterpret_cast<const unsigned char *>(dinp) +
+                                      row0 * row_bytes,
+                                  bytes, bar);
                 });
         }
     } else {
         const int64_t rstep = tstep * RT;
         int64_t r = tile0 * RT + group;
         float m_next = 0.f, s_next = 0.f;
-        if (ntiles_here > 0 && r < N) {
+        if (!RECOMP && ntiles_here > 0 && r < N) {
             m_next = __ldg(mean + r);
             s_next = __ldg(rstd + r);
         }
@@ -429,14 +300,15 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 if constexpr (W == 1) break;
             }
             const bool valid = r < N;                 // uniform over the row group
-            const float m = m_next, s = s_next;
-            if (k + 1 < ntiles_here && r + rstep < N) {   // next row's statistics
+            float m = m_next, s = s_next;
+            if (!RECOMP && k + 1 < ntiles_here && r + rstep < N) {   // next row's statistics
                 m_next = __ldg(mean + r + rstep);
                 s_next = __ldg(rstd + r + rstep);
             }
             const unsigned char *stage = ring + size_t(st) * stage_bytes + group * row_bytes;
             const uint4 *xs = reinterpret_cast<const uint4 *>(stage);
             const uint4 *ds = reinterpret_cast<const uint4 *>(stage + half_bytes);
+            const uint4 *ps = reinterpret_cast<const uint4 *>(stage + 2 * half_bytes);
             uint4 xv[V], dv[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
@@ -445,34 +317,91 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 xv[i] = ok ? xs[j] : make_uint4(0u, 0u, 0u, 0u);
                 dv[i] = ok ? ds[j] : make_uint4(0u, 0u, 0u, 0u);
             }
-            fence_proxy_async_smem();                 // reads done before the refill
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-            if (!valid) continue;
-            float *slot = s_red + (group * 2 + parity) * 3 * W;
-            parity ^= 1;
+            const float pivot = (RECOMP && valid) ? to_f32(reinterpret_cast<const T *>(stage)[0])
+                                                  : 0.f;
+            // Release the stage once this warp's reads of it are done: right
+            // away, or after pass 2 when it also holds the previous dinp.
+            auto release = [&]() {
+                fence_proxy_async_smem();             // reads done before the refill
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            };
+            if constexpr (!ACC) release();
+            if (!valid) {
+                if constexpr (ACC) release();
+                continue;
+            }
 
             // Pass 1 / pass 2.  Where the register budget allows (KEEP_D), pass 1
             // keeps d = x - mean as fp32 pairs and pass 2 evaluates
             //   dinp = g*rstd + NA + d*NC,  NA = -rstd*mean(g),
             //   NC = -rstd^3*mean(g*d)   (xhat = d*rstd),
             // so pass 2 never unpacks x again; otherwise both passes rebuild
-            // xhat from the packed row.
+            // xhat from the packed row.  Recomputing the statistics, d is
+            // (x - pivot) - mean(x - pivot) and K, MD below are the pivot and
+            // that mean; from the saved statistics K = mean[r] and MD = 0.
             constexpr bool KEEP_D = sizeof(T) == 4 || V <= 3;
             uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
-            const f32x2 M = pair(m, m);
-            const f32x2 Sx = pair(s, s);
             f32x2 d[KEEP_D ? V : 1][P];
+            f32x2 K = pair(m, m), MD = pair(0.f, 0.f);
+            if constexpr (RECOMP) {
+                K = pair(pivot, pivot);
+                f32x2 sd = pair(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const bool in = t + TPR * i < nvec;
+                    f32x2 x[P];
+                    to_pairs(xv[i], x);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        const f32x2 dq = sub2(x[q], K);
+                        if constexpr (KEEP_D) d[i][q] = dq;
+                        if (in) sd = add2(sd, dq);
+                    }
+                }
+                float a = warp_sum(hsum(sd)), unused = 0.f;
+                abort = group_exchange<W>(a, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                                          group, sub, lane);
+                parity ^= 1;
+                const float md = a * inv_C;
+                MD = pair(md, md);
+                f32x2 sq = pair(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const bool in = t + TPR * i < nvec;
+                    f32x2 x[P];
+                    if constexpr (!KEEP_D) to_pairs(xv[i], x);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        f32x2 dq;
+                        if constexpr (KEEP_D) {
+                            d[i][q] = sub2(d[i][q], MD);
+                            dq = d[i][q];
+                        } else {
+                            dq = sub2(sub2(x[q], K), MD);
+                        }
+                        if (in) sq = fma2(dq, dq, sq);
+                    }
+                }
+                float v = warp_sum(hsum(sq));
+                abort = group_exchange<W>(v, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                                          group, sub, lane);
+                parity ^= 1;
+                s = rsqrtf(v * inv_C + eps);
+            }
+            float *slot = s_red + (group * 2 + parity) * 3 * W;
+            parity ^= 1;
+            const f32x2 Sx = pair(s, s);
             f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int j = t + TPR * i;
-                if constexpr (KEEP_D) {
+                if constexpr (KEEP_D && !RECOMP) {
                     // d for every slot (dead lanes' values are never used)
                     f32x2 dq[P];
                     to_pairs(xv[i], dq);
 #pragma unroll
-                    for (int q = 0; q < P; ++q) d[i][q] = sub2(dq[q], M);
+                    for (int q = 0; q < P; ++q) d[i][q] = sub2(dq[q], K);
                 }
                 if (j < nvec) {
                     f32x2 dy[P], wp[P];
@@ -490,7 +419,9 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                         to_pairs(xv[i], x);
 #pragma unroll
                         for (int q = 0; q < P; ++q) {
-                            const f32x2 xh = mul2(sub2(x[q], M), Sx);
+                            f32x2 dq = sub2(x[q], K);
+                            if constexpr (RECOMP) dq = sub2(dq, MD);
+                            const f32x2 xh = mul2(dq, Sx);
                             const f32x2 g = mul2(dy[q], wp[q]);
                             s1 = add2(s1, g);
                             s2 = fma2(g, xh, s2);                 // sum g * xhat
@@ -520,15 +451,24 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                             o[q] = fma2(g, Sx, fma2(d[i][q], NCc, NA));
                             xh = mul2(d[i][q], Sx);
                         } else {
-                            xh = mul2(sub2(pair_at<T>(xv[i], q), M), Sx);
+                            f32x2 dq = sub2(pair_at<T>(xv[i], q), K);
+                            if constexpr (RECOMP) dq = sub2(dq, MD);
+                            xh = mul2(dq, Sx);
                             o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
                         }
                         acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
                         acc_b[i][q] = add2(acc_b[i][q], dy);
                     }
+                    if constexpr (ACC) {
+                        f32x2 pp[P];
+                        to_pairs(ps[j], pp);
+#pragma unroll
+                        for (int q = 0; q < P; ++q) o[q] = add2(o[q], pp[q]);
+                    }
                     __stcs(gr + j, from_pairs(o));
                 }
             }
+            if constexpr (ACC) release();
             if (abort) break;                         // the whole row group leaves here
         }
     }

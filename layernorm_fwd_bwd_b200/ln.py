@@ -28,6 +28,10 @@ LN_ERR_EPS = 4
 LN_ERR_WORKSPACE = 5
 LN_ERR_CUDA = 6
 LN_ERR_SCRATCH = 7
+LN_ERR_FLAGS = 8
+LN_BWD_ACCUMULATE_DINP = 1
+LN_BWD_ACCUMULATE_DPARAMS = 2
+LN_BWD_RECOMPUTE_STATS = 4
 LN_NOALLOC_SCRATCH_BYTES = 4 << 20
 LN_NOALLOC_MAX_C = LN_NOALLOC_SCRATCH_BYTES // 8
 
@@ -45,6 +49,12 @@ _lib.ln_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
 _lib.ln_backward_noalloc.restype = _int
 _lib.ln_backward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                      _int, _vp]
+_lib.ln_forward_residual.restype = _int
+_lib.ln_forward_residual.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32,
+                                     _int, _vp]
+_lib.ln_backward_ex.restype = _int
+_lib.ln_backward_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _int,
+                                ctypes.c_uint, _vp]
 _lib.ln_status_string.restype = ctypes.c_char_p
 _lib.ln_status_string.argtypes = [_int]
 _lib.ln_launch_count.restype = ctypes.c_uint64
@@ -123,6 +133,27 @@ def ln_backward(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
                             int(N), int(C), int(dtype), _stream(stream)))
 
 
+def ln_forward_residual(resid_out, out, mean, rstd, resid, branch, weight, bias, N: int,
+                        C: int, eps: float, dtype: int, stream=None) -> None:
+    """resid_out <- resid + branch (rounded to dtype); out, mean, rstd <-
+    LayerNorm(resid_out; weight, bias, eps).  No output may overlap an
+    input."""
+    _check(_lib.ln_forward_residual(_ptr(resid_out), _ptr(out), _ptr(mean), _ptr(rstd),
+                                    _ptr(resid), _ptr(branch), _ptr(weight), _ptr(bias),
+                                    int(N), int(C), float(eps), int(dtype), _stream(stream)))
+
+
+def ln_backward_ex(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int, C: int,
+                   eps: float, dtype: int, flags: int, stream=None) -> None:
+    """ln_backward with variants selected by ``flags`` (LN_BWD_ACCUMULATE_DINP:
+    dinp +=; LN_BWD_ACCUMULATE_DPARAMS: dweight/dbias +=;
+    LN_BWD_RECOMPUTE_STATS: mean/rstd recomputed from inp with eps, so they
+    may be None)."""
+    _check(_lib.ln_backward_ex(_ptr(dinp), _ptr(dweight), _ptr(dbias), _ptr(dout),
+                               _ptr(inp), _ptr(weight), _ptr(mean), _ptr(rstd), int(N),
+                               int(C), float(eps), int(dtype), int(flags), _stream(stream)))
+
+
 def ln_backward_noalloc(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
                         C: int, dtype: int, stream=None) -> None:
     """ln_backward for callers that cannot allocate device memory: its partial
@@ -143,3 +174,14 @@ def raw_forward(*args) -> int:
 def raw_backward(*args) -> int:
     """Call ln_backward with already-marshalled arguments; returns the status."""
     return int(_lib.ln_backward(*args))
+
+
+def raw_forward_residual(*args) -> int:
+    """Call ln_forward_residual with already-marshalled arguments; returns the
+    status."""
+    return int(_lib.ln_forward_residual(*args))
+
+
+def raw_backward_ex(*args) -> int:
+    """Call ln_backward_ex with already-marshalled arguments; returns the status."""
+    return int(_lib.ln_backward_ex(*args))

@@ -39,6 +39,12 @@ def nan_tensor(shape, tdtype, device="cuda") -> torch.Tensor:
     return torch.full(shape, float("nan"), dtype=tdtype, device=device)
 
 
+def forward_outputs(N, C, dtype):
+    """NaN-filled out, mean, rstd (so an element the library skips shows)."""
+    return (nan_tensor((N, C), TORCH_DT[dtype]), nan_tensor((N,), torch.float32),
+            nan_tensor((N,), torch.float32))
+
+
 def forward(lib, inp, w, b, N, C, eps, dtype, stream=None):
     out = nan_tensor((N, C), TORCH_DT[dtype])
     mean = nan_tensor((N,), torch.float32)
@@ -66,3 +72,9 @@ def full_batch(name: str) -> wl.Batch:
     """The named workload at its full size (cached: drawing 50M elements takes
     seconds)."""
     return wl.generate(wl.WORKLOADS[name])
+
+
+@functools.lru_cache(maxsize=2)
+def full_extras(name: str) -> wl.Extras:
+    """The variants' extra inputs for the named workload at full size."""
+    return wl.generate_extras(wl.WORKLOADS[name])

@@ -44,12 +44,13 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
-        assert lib.ln_status_string(code).startswith(
-            ["LN_OK", "LN_ERR_NULL", "LN_ERR_SHAPE", "LN_ERR_DTYPE", "LN_ERR_EPS",
-             "LN_ERR_WORKSPACE", "LN_ERR_CUDA"][code])
+    names = ["LN_OK", "LN_ERR_NULL", "LN_ERR_SHAPE", "LN_ERR_DTYPE", "LN_ERR_EPS",
+             "LN_ERR_WORKSPACE", "LN_ERR_CUDA", "LN_ERR_SCRATCH", "LN_ERR_FLAGS"]
+    for code, name in enumerate(names):
+        assert lib.ln_status_string(code).startswith(name)
+        assert getattr(lib, name) == code
     assert lib.ln_status_string(99) == "unknown ln_status"
-    assert lib.version() == 1
+    assert lib.version() == 2
 
 
 def test_host_validation_without_gpu(lib):
@@ -72,6 +73,39 @@ def test_host_validation_without_gpu(lib):
     assert b(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 7, None) == lib.LN_ERR_DTYPE
     assert b(nz, None, nz, nz, nz, nz, nz, nz, 4, 8, 0, None) == lib.LN_ERR_NULL
     assert b(nz, nz, None, nz, nz, nz, nz, nz, 0, 8, 0, None) == lib.LN_ERR_NULL
+    assert lib.launch_count() == 0
+
+
+def test_variant_validation_without_gpu(lib):
+    # ln_forward_residual and ln_backward_ex validate like the plain calls,
+    # plus their own arguments, before any CUDA call.
+    nz = 16
+    r = lib.raw_forward_residual
+    assert r(nz, nz, nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, None) == lib.LN_ERR_SHAPE
+    assert r(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 5, None) == lib.LN_ERR_DTYPE
+    assert r(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 0.0, 0, None) == lib.LN_ERR_EPS
+    assert r(None, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 0, None) == lib.LN_ERR_NULL
+    assert r(nz, nz, nz, nz, nz, None, nz, nz, 4, 8, 1e-5, 0, None) == lib.LN_ERR_NULL
+    assert r(nz, None, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 1, None) == lib.LN_ERR_NULL
+    assert r(None, None, None, None, None, None, None, None, 0, 8, 1e-5, 0, None) == lib.LN_OK
+    x = lib.raw_backward_ex
+    acc = lib.LN_BWD_ACCUMULATE_DINP | lib.LN_BWD_ACCUMULATE_DPARAMS
+    rec = lib.LN_BWD_RECOMPUTE_STATS
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, 0, None) == lib.LN_ERR_SHAPE
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 3, 0, None) == lib.LN_ERR_DTYPE
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 0, 8, None) == lib.LN_ERR_FLAGS
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 0, 1 << 31, None) == lib.LN_ERR_FLAGS
+    # eps is checked only when the statistics are recomputed
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 0.0, 0, rec, None) == lib.LN_ERR_EPS
+    assert x(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, float("nan"), 1, rec | acc,
+             None) == lib.LN_ERR_EPS
+    # mean/rstd are required unless recomputed
+    assert x(nz, nz, nz, nz, nz, nz, None, nz, 4, 8, 1e-5, 0, acc, None) == lib.LN_ERR_NULL
+    assert x(nz, nz, nz, nz, nz, nz, nz, None, 4, 8, 1e-5, 0, 0, None) == lib.LN_ERR_NULL
+    assert x(nz, None, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 0, rec, None) == lib.LN_ERR_NULL
+    # N == 0 with accumulated parameters has nothing to do (no memset either)
+    assert x(None, nz, nz, None, None, None, None, None, 0, 8, 0.0, 0,
+             lib.LN_BWD_ACCUMULATE_DPARAMS, None) == lib.LN_OK
     assert lib.launch_count() == 0
 
 
