@@ -71,7 +71,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-variants", action="store_true",
-                   help="skip timing ln_forward_residual and ln_backward_ex")
+                   help="skip timing ln_forward_residual, ln_backward_ex and fp16")
     p.add_argument("--sets", type=int, default=SETS,
                    help="rotating buffer sets (>= 2 so a step's backward never "
                         "reads what its forward just read)")
@@ -392,7 +392,8 @@ def run_variants(torch, ln, stream, sets, weight, bias, dweight, dbias, w, eps, 
     (inputs never re-read from L2), timed with CUDA events around the loop on
     the launching stream.  The inputs reuse the sets' arrays (a branch is
     another set's dout; accumulation goes into whatever dinp holds), which
-    changes no byte counts."""
+    changes no byte counts.  For a 16-bit workload, plain forward and
+    backward also run on fp16 copies of the sets."""
     N, C = w.N, w.C
     n = len(sets)
     sp = stream.cuda_stream
@@ -425,9 +426,32 @@ def run_variants(torch, ln, stream, sets, weight, bias, dweight, dbias, w, eps, 
                 raise ln.LNError(rc)
         return run
 
-    for name, call in (("fwd_residual", fwd_res), ("bwd_accumulate", bwd_ex(acc)),
-                       ("bwd_recompute", bwd_ex(rec)),
-                       ("bwd_accumulate_recompute", bwd_ex(acc | rec))):
+    cases = [("fwd_residual", fwd_res), ("bwd_accumulate", bwd_ex(acc)),
+             ("bwd_recompute", bwd_ex(rec)), ("bwd_accumulate_recompute", bwd_ex(acc | rec))]
+    if w.elem_bytes == 2:
+        # the same shape with fp16 activations (the sets' values converted)
+        with torch.cuda.stream(stream):
+            h = [{k: (v.to(torch.float16) if v.dtype == torch.bfloat16 else torch.empty_like(v))
+                  for k, v in st.items()} for st in sets]
+            hw, hb = weight.to(torch.float16), bias.to(torch.float16)
+        f16 = ln.LN_F16
+
+        def h_fwd(i):
+            a = h[i % n]
+            return ln.raw_forward(ptr(a["out"]), ptr(a["mean"]), ptr(a["rstd"]), ptr(a["inp"]),
+                                  ptr(hw), ptr(hb), N, C, eps, f16, sp)
+
+        def h_bwd(i):
+            b = h[i % n]
+            return ln.raw_backward(ptr(b["dinp"]), ptr(dweight), ptr(dbias), ptr(b["dout"]),
+                                   ptr(b["inp"]), ptr(hw), ptr(b["mean"]), ptr(b["rstd"]), N, C,
+                                   f16, sp)
+
+        for k in range(n):                  # statistics for every fp16 set
+            checked(h_fwd)(k)
+        nbytes["fp16_fwd"], nbytes["fp16_bwd"] = w.fwd_bytes(), w.bwd_bytes()
+        cases += [("fp16_fwd", h_fwd), ("fp16_bwd", h_bwd)]
+    for name, call in cases:
         us = call_loop_us(torch, stream, checked(call), calls)
         gbs = nbytes[name] / (us * 1e-6) / 1e9
         out[name] = {"us": round(us, 3), "GB_s": round(gbs, 1), "bytes": nbytes[name],

@@ -25,9 +25,12 @@
  * C elements, mean and rstd hold N.  All pointers are DEVICE pointers of the
  * current CUDA device, owned by the caller; the library never frees them.
  *
- * Types.  `dtype` (LN_F32 or LN_BF16) is the element type of inp, out, dout,
- * dinp, weight and bias.  mean, rstd, dweight and dbias are always fp32.
- * Arithmetic is fp32 in registers; bf16 results are rounded to nearest-even.
+ * Types.  `dtype` (LN_F32, LN_BF16 or LN_F16) is the element type of inp,
+ * out, dout, dinp, weight and bias.  mean, rstd, dweight and dbias are always
+ * fp32.  Arithmetic is fp32 in registers; bf16 and fp16 results are rounded
+ * to nearest-even (fp16 results beyond 65504 become infinite, as rounding
+ * requires).  The pages this library follows name fp32 and bf16 kernels;
+ * fp16 is the other 16-bit training format and takes the same paths.
  *
  * Semantics shared by every call.
  *   - Asynchronous on `stream` (NULL: the legacy default stream); no host
@@ -65,7 +68,8 @@ typedef struct CUstream_st *ln_stream_t;
 
 typedef enum {
     LN_F32 = 0,   /* IEEE binary32 */
-    LN_BF16 = 1   /* bfloat16 (8 significant bits, binary32 exponent range) */
+    LN_BF16 = 1,  /* bfloat16 (8 significant bits, binary32 exponent range) */
+    LN_F16 = 2    /* IEEE binary16 (11 significant bits, largest finite 65504) */
 } ln_dtype;
 
 typedef enum {
@@ -73,7 +77,7 @@ typedef enum {
     LN_ERR_NULL = 1,       /* a required pointer is NULL */
     LN_ERR_SHAPE = 2,      /* N < 0, N > LN_MAX_N, C < 1, C > LN_MAX_C or
                               N * C > LN_MAX_ELEMS */
-    LN_ERR_DTYPE = 3,      /* dtype is not LN_F32 or LN_BF16 */
+    LN_ERR_DTYPE = 3,      /* dtype is not LN_F32, LN_BF16 or LN_F16 */
     LN_ERR_EPS = 4,        /* eps is not finite, or not > 0 */
     LN_ERR_WORKSPACE = 5,  /* the backward's workspace could not be allocated */
     LN_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
@@ -221,7 +225,8 @@ uint64_t ln_launch_count(void);
  * the current device.  Returns LN_OK, LN_ERR_NULL or LN_ERR_CUDA. */
 int ln_device_status(unsigned int *bits, int clear);
 
-/* Library ABI version: 2 (1 plus ln_forward_residual and ln_backward_ex). */
+/* Library ABI version: 2 (1 plus ln_forward_residual, ln_backward_ex and
+ * LN_F16). */
 int ln_version(void);
 
 #ifdef __cplusplus

@@ -25,10 +25,10 @@ BUILD_DIR = os.path.join(PKG, "_build")
 LIBRARY = os.path.join(PKG, "libln.so")
 
 # (direction, element type, variant): direction 0 forward / 1 backward;
-# type 0 fp32 / 1 bf16; forward variants 0 plain / 1 residual, backward
-# variants bit 0 accumulate dinp, bit 1 recompute the statistics.
-INSTANCES = [(0, t, m) for t in (0, 1) for m in (0, 1)] + \
-            [(1, t, m) for t in (0, 1) for m in (0, 1, 2, 3)]
+# type 0 fp32 / 1 bf16 / 2 fp16; forward variants 0 plain / 1 residual,
+# backward variants bit 0 accumulate dinp, bit 1 recompute the statistics.
+INSTANCES = [(0, t, m) for t in (0, 1, 2) for m in (0, 1)] + \
+            [(1, t, m) for t in (0, 1, 2) for m in (0, 1, 2, 3)]
 UNITS = ["ln_api.cu", "ln_noalloc.cu"]
 DEPENDS = [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))
            if f.endswith((".cu", ".cuh"))] + [os.path.join(INCLUDE, "ln.h")]

@@ -89,7 +89,7 @@ int check_shape(int64_t N, int64_t C) {
     return LN_OK;
 }
 
-bool valid_dtype(int dtype) { return dtype == LN_F32 || dtype == LN_BF16; }
+bool valid_dtype(int dtype) { return dtype == LN_F32 || dtype == LN_BF16 || dtype == LN_F16; }
 bool valid_eps(float eps) { return std::isfinite(eps) && eps > 0.f; }
 
 template <typename T>
@@ -124,7 +124,11 @@ int forward_entry(void *out, float *mean, float *rstd, const void *inp, const vo
                          weight,    bias,       resid_out,      branch,
                          N,         (int)C,     1.0f / float(C), eps,
                          reinterpret_cast<cudaStream_t>(stream), dev, ds->sms, ds->status};
-    return dtype == LN_F32 ? fwd_call<float>(a, residual) : fwd_call<lnk::bf16>(a, residual);
+    switch (dtype) {
+        case LN_F32: return fwd_call<float>(a, residual);
+        case LN_BF16: return fwd_call<lnk::bf16>(a, residual);
+        default: return fwd_call<lnk::f16>(a, residual);
+    }
 }
 
 }  // namespace
@@ -179,7 +183,11 @@ int backward_entry(void *dinp, float *dweight, float *dbias, const void *dout,
                     ds->sms,       ds->pool,  scratch,  scratch_floats, ds->status};
     const int mode = ((flags & LN_BWD_ACCUMULATE_DINP) ? lnk::kBwdAccumulate : 0) |
                      (recompute ? lnk::kBwdRecompute : 0);
-    return dtype == LN_F32 ? bwd_call<float>(a, mode) : bwd_call<lnk::bf16>(a, mode);
+    switch (dtype) {
+        case LN_F32: return bwd_call<float>(a, mode);
+        case LN_BF16: return bwd_call<lnk::bf16>(a, mode);
+        default: return bwd_call<lnk::f16>(a, mode);
+    }
 }
 
 }  // namespace lnh
@@ -221,7 +229,7 @@ const char *ln_status_string(int status) {
         case LN_OK: return "LN_OK: success";
         case LN_ERR_NULL: return "LN_ERR_NULL: a required pointer is NULL";
         case LN_ERR_SHAPE: return "LN_ERR_SHAPE: N or C out of range (0 <= N <= 2^40, 1 <= C <= 2^24, N*C <= 2^50)";
-        case LN_ERR_DTYPE: return "LN_ERR_DTYPE: dtype must be LN_F32 (0) or LN_BF16 (1)";
+        case LN_ERR_DTYPE: return "LN_ERR_DTYPE: dtype must be LN_F32 (0), LN_BF16 (1) or LN_F16 (2)";
         case LN_ERR_EPS: return "LN_ERR_EPS: eps must be finite and > 0";
         case LN_ERR_WORKSPACE: return "LN_ERR_WORKSPACE: backward workspace allocation failed";
         case LN_ERR_CUDA: return "LN_ERR_CUDA: a CUDA runtime call or kernel launch failed";

@@ -121,7 +121,7 @@ struct BwdArgs {
     unsigned int *status;
 };
 
-// Instantiated in ln_inst.cu for T in {float, bf16} and every MODE (see
+// Instantiated in ln_inst.cu for T in {float, bf16, f16} and every MODE (see
 // lnk::kFwdResidual, lnk::kBwdAccumulate, lnk::kBwdRecompute).
 template <typename T, int MODE>
 int fwd_dispatch(const FwdArgs &a);

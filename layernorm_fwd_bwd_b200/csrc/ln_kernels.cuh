@@ -31,61 +31,32 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace lnk {
 
 using bf16 = __nv_bfloat16;
+using f16 = __half;
 
 // Elements per 16-byte vector.
 template <typename T> struct Vec;
 template <> struct Vec<float> { static constexpr int E = 4; };
 template <> struct Vec<bf16> { static constexpr int E = 8; };
-
-__device__ __forceinline__ void unpack(const uint4 &v, float (&f)[4]) {
-    f[0] = __uint_as_float(v.x);
-    f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z);
-    f[3] = __uint_as_float(v.w);
-}
-
-// bf16 element 2k sits in the low half of word k (little endian); widening a
-// bf16 to fp32 is placing its 16 bits in the high half of a word.
-__device__ __forceinline__ void unpack(const uint4 &v, float (&f)[8]) {
-    f[0] = __uint_as_float(v.x << 16);
-    f[1] = __uint_as_float(v.x & 0xffff0000u);
-    f[2] = __uint_as_float(v.y << 16);
-    f[3] = __uint_as_float(v.y & 0xffff0000u);
-    f[4] = __uint_as_float(v.z << 16);
-    f[5] = __uint_as_float(v.z & 0xffff0000u);
-    f[6] = __uint_as_float(v.w << 16);
-    f[7] = __uint_as_float(v.w & 0xffff0000u);
-}
-
-__device__ __forceinline__ uint4 pack(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
-                      __float_as_uint(f[2]), __float_as_uint(f[3]));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);   // round to nearest-even
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ uint4 pack(const float (&f)[8]) {
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-}
+template <> struct Vec<f16> { static constexpr int E = 8; };
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(f16 v) { return __half2float(v); }
 
+// fp32 -> T, rounded to nearest-even.
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) {
     return __float2bfloat16_rn(v);
 }
+template <> __device__ __forceinline__ f16 from_f32<f16>(float v) { return __float2half_rn(v); }
 
 // Butterfly all-reduce: every lane ends with the same bits (each level adds
 // the same two values, in either order).
@@ -184,16 +155,39 @@ __device__ __forceinline__ float hsum(f32x2 v) {
     return lo + hi;
 }
 
-// A 16-byte vector as P = E/2 pairs, and back (bf16 rounded to nearest-even).
-__device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[2]) {
+// A 16-byte vector of T as P = E/2 fp32 pairs, and back (bf16 and fp16
+// rounded to nearest-even).  Element 2k of a 16-bit vector sits in the low
+// half of word k (little endian).  Widening a bf16 is placing its 16 bits in
+// the high half of a word; fp16 takes the hardware conversion.
+template <typename T>
+__device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[Vec<T>::E / 2]);
+template <>
+__device__ __forceinline__ void to_pairs<float>(const uint4 &v, f32x2 (&p)[2]) {
     p[0] = pair(__uint_as_float(v.x), __uint_as_float(v.y));
     p[1] = pair(__uint_as_float(v.z), __uint_as_float(v.w));
 }
-__device__ __forceinline__ void to_pairs(const uint4 &v, f32x2 (&p)[4]) {
-    p[0] = pair(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
-    p[1] = pair(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-    p[2] = pair(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
-    p[3] = pair(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+__device__ __forceinline__ f32x2 bf16x2_pair(uint32_t w) {
+    return pair(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ f32x2 f16x2_pair(uint32_t w) {
+    __half2 h;
+    memcpy(&h, &w, 4);
+    const float2 f = __half22float2(h);
+    return pair(f.x, f.y);
+}
+template <>
+__device__ __forceinline__ void to_pairs<bf16>(const uint4 &v, f32x2 (&p)[4]) {
+    p[0] = bf16x2_pair(v.x);
+    p[1] = bf16x2_pair(v.y);
+    p[2] = bf16x2_pair(v.z);
+    p[3] = bf16x2_pair(v.w);
+}
+template <>
+__device__ __forceinline__ void to_pairs<f16>(const uint4 &v, f32x2 (&p)[4]) {
+    p[0] = f16x2_pair(v.x);
+    p[1] = f16x2_pair(v.y);
+    p[2] = f16x2_pair(v.z);
+    p[3] = f16x2_pair(v.w);
 }
 // Pair q of a 16-byte vector (q < E/2), unpacked on its own.
 template <typename T>
@@ -203,24 +197,51 @@ __device__ __forceinline__ f32x2 pair_at<float>(const uint4 &v, int q) {
     return q == 0 ? pair(__uint_as_float(v.x), __uint_as_float(v.y))
                   : pair(__uint_as_float(v.z), __uint_as_float(v.w));
 }
+__device__ __forceinline__ uint32_t word_at(const uint4 &v, int q) {
+    return q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
+}
 template <>
 __device__ __forceinline__ f32x2 pair_at<bf16>(const uint4 &v, int q) {
-    const uint32_t w = q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
-    return pair(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    return bf16x2_pair(word_at(v, q));
 }
-__device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[2]) {
+template <>
+__device__ __forceinline__ f32x2 pair_at<f16>(const uint4 &v, int q) {
+    return f16x2_pair(word_at(v, q));
+}
+template <typename T>
+__device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[Vec<T>::E / 2]);
+template <>
+__device__ __forceinline__ uint4 from_pairs<float>(const f32x2 (&p)[2]) {
     float a, b, c, d;
     split(p[0], a, b);
     split(p[1], c, d);
     return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c),
                       __float_as_uint(d));
 }
-__device__ __forceinline__ uint4 from_pairs(const f32x2 (&p)[4]) {
-    float f[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) split(p[k], f[2 * k], f[2 * k + 1]);
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+__device__ __forceinline__ uint32_t pack_bf16x2(f32x2 v) {
+    float lo, hi;
+    split(v, lo, hi);
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);   // round to nearest-even
+    uint32_t w;
+    memcpy(&w, &h, 4);
+    return w;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(f32x2 v) {
+    float lo, hi;
+    split(v, lo, hi);
+    __half2 h = __floats2half2_rn(lo, hi);              // round to nearest-even
+    uint32_t w;
+    memcpy(&w, &h, 4);
+    return w;
+}
+template <>
+__device__ __forceinline__ uint4 from_pairs<bf16>(const f32x2 (&p)[4]) {
+    return make_uint4(pack_bf16x2(p[0]), pack_bf16x2(p[1]), pack_bf16x2(p[2]),
+                      pack_bf16x2(p[3]));
+}
+template <>
+__device__ __forceinline__ uint4 from_pairs<f16>(const f32x2 (&p)[4]) {
+    return make_uint4(pack_f16x2(p[0]), pack_f16x2(p[1]), pack_f16x2(p[2]), pack_f16x2(p[3]));
 }
 // P pairs of fp32 values from shared memory (16-byte aligned address).
 template <int P>
@@ -248,29 +269,20 @@ constexpr int kBwdAccumulate = 1;
 // pivot-shifted two-pass statistics instead of being read from the arrays.
 constexpr int kBwdRecompute = 2;
 
-// a + b elementwise for two 16-byte vectors of T, each sum rounded to T
-// (fp32: the sum itself; bf16: the fp32 sum is exact or rounds far from a
-// bf16 rounding boundary, so rounding it to nearest-even gives the correctly
-// rounded bf16 sum).
-__device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b, float) {
-    f32x2 pa[2], pb[2];
-    to_pairs(a, pa);
-    to_pairs(b, pb);
-    pa[0] = add2(pa[0], pb[0]);
-    pa[1] = add2(pa[1], pb[1]);
-    return from_pairs(pa);
-}
-__device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b, bf16) {
-    f32x2 pa[4], pb[4];
-    to_pairs(a, pa);
-    to_pairs(b, pb);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) pa[q] = add2(pa[q], pb[q]);
-    return from_pairs(pa);
-}
+// a + b elementwise for two 16-byte vectors of T, each sum rounded to T.
+// fp32: the sum itself.  bf16 / fp16: the fp32 sum of two such values is
+// exact, or (operands far apart in magnitude) within half an fp32 ulp of a
+// value that is far from any bf16 / fp16 rounding boundary, so rounding it to
+// nearest-even gives the correctly rounded sum.
 template <typename T>
 __device__ __forceinline__ uint4 add_round(const uint4 &a, const uint4 &b) {
-    return add_round(a, b, T());
+    constexpr int P = Vec<T>::E / 2;
+    f32x2 pa[P], pb[P];
+    to_pairs<T>(a, pa);
+    to_pairs<T>(b, pb);
+#pragma unroll
+    for (int q = 0; q < P; ++q) pa[q] = add2(pa[q], pb[q]);
+    return from_pairs<T>(pa);
 }
 // One element of the rounded sum (same value as the vector form).
 template <typename T>
@@ -411,7 +423,7 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
         if constexpr (W == 1) {
             float lo, hi;
             f32x2 p0[P];
-            to_pairs(xv[0], p0);            // lane 0 holds columns 0 .. E-1
+            to_pairs<T>(xv[0], p0);            // lane 0 holds columns 0 .. E-1
             split(p0[0], lo, hi);
             pivot = __shfl_sync(0xffffffffu, lo, 0);
         } else if constexpr (RES) {
@@ -426,7 +438,7 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const bool ok = t + i * TPR < nvec;
-            to_pairs(xv[i], d[i]);
+            to_pairs<T>(xv[i], d[i]);
 #pragma unroll
             for (int k = 0; k < P; ++k) {
                 d[i][k] = sub2(d[i][k], K);
@@ -460,7 +472,7 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
                 smem_pairs<P>(s_b + j * E, bp);
 #pragma unroll
                 for (int k = 0; k < P; ++k) o[k] = fma2(mul2(d[i][k], R), wp[k], bp[k]);
-                __stcs(yr + j, from_pairs(o));
+                __stcs(yr + j, from_pairs<T>(o));
             }
         }
         if (t == 0) {
@@ -550,7 +562,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             if constexpr (W == 1) {
                 float lo, hi;
                 f32x2 p0[P];
-                to_pairs(xv[0], p0);        // lane 0 holds columns 0 .. E-1
+                to_pairs<T>(xv[0], p0);        // lane 0 holds columns 0 .. E-1
                 split(p0[0], lo, hi);
                 pivot = __shfl_sync(0xffffffffu, lo, 0);
             } else {
@@ -562,7 +574,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             for (int i = 0; i < V; ++i) {
                 if (t + i * TPR < nvec) {
                     f32x2 x[P];
-                    to_pairs(xv[i], x);
+                    to_pairs<T>(xv[i], x);
 #pragma unroll
                     for (int k = 0; k < P; ++k) sd = add2(sd, sub2(x[k], K));
                 }
@@ -576,7 +588,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             for (int i = 0; i < V; ++i) {
                 if (t + i * TPR < nvec) {
                     f32x2 x[P];
-                    to_pairs(xv[i], x);
+                    to_pairs<T>(xv[i], x);
 #pragma unroll
                     for (int k = 0; k < P; ++k) {
                         const f32x2 d = sub2(sub2(x[k], K), MD);
@@ -606,8 +618,8 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             const int j = t + i * TPR;
             if (j < nvec) {
                 f32x2 x[P], dy[P], wp[P];
-                to_pairs(xv[i], x);
-                to_pairs(dv[i], dy);
+                to_pairs<T>(xv[i], x);
+                to_pairs<T>(dv[i], dy);
                 smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
                 for (int k = 0; k < P; ++k) {
@@ -631,8 +643,8 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             const int j = t + i * TPR;
             if (j < nvec) {
                 f32x2 x[P], dy[P], wp[P], o[P];
-                to_pairs(xv[i], x);
-                to_pairs(dv[i], dy);
+                to_pairs<T>(xv[i], x);
+                to_pairs<T>(dv[i], dy);
                 smem_pairs<P>(s_w + j * E, wp);
 #pragma unroll
                 for (int k = 0; k < P; ++k) {
@@ -644,11 +656,11 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 }
                 if constexpr (ACC) {
                     f32x2 pp[P];
-                    to_pairs(__ldcs(gr + j), pp);
+                    to_pairs<T>(__ldcs(gr + j), pp);
 #pragma unroll
                     for (int k = 0; k < P; ++k) o[k] = add2(o[k], pp[k]);
                 }
-                __stcs(gr + j, from_pairs(o));
+                __stcs(gr + j, from_pairs<T>(o));
             }
         }
     }

@@ -63,7 +63,7 @@ extern "C" int ln_backward_noalloc(void *dinp, float *dweight, float *dbias,
                                    int64_t C, int dtype, ln_stream_t stream) {
     if (N < 0 || N > LN_MAX_N || C < 1 || C > LN_MAX_C || N > LN_MAX_ELEMS / C)
         return LN_ERR_SHAPE;
-    if (dtype != LN_F32 && dtype != LN_BF16) return LN_ERR_DTYPE;
+    if (dtype != LN_F32 && dtype != LN_BF16 && dtype != LN_F16) return LN_ERR_DTYPE;
     if (C > LN_NOALLOC_MAX_C) return LN_ERR_SCRATCH;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LN_ERR_CUDA;

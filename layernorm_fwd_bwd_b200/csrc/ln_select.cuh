@@ -6,7 +6,7 @@
 // (ln_tile.cuh): one warp per row up to 4 vectors, two warps per row for 5..8;
 // wider rows take the persistent register-resident kernel with W = 4, 8 or 16
 // warps per row and 4 vectors per thread.
-// Backward: rows of up to 4 (bf16) / 6 (fp32) vectors per lane take the
+// Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
 // persistent TMA-ring kernel (ln_tma.cuh) on one warp per row, wider rows the
 // ring with W = 2..4 warps per row; rows wider than that take the
 // register-resident kernel (W = 4..16 warps per row, 4 vectors per thread).
@@ -117,13 +117,12 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
 // stages of the widest rows still fit in shared memory; recomputing the
 // statistics, bf16 rows of 4 vectors per lane would spill, so they go to two
 // warps.
-template <typename T, int MODE> struct RingVmax;
+template <typename T, int MODE> struct RingVmax {   // 16-bit elements (bf16, fp16)
+    static constexpr int one = (MODE & kBwdRecompute) ? 3 : 4, shared = 3;
+};
 template <int MODE> struct RingVmax<float, MODE> {
     static constexpr bool kAcc = (MODE & kBwdAccumulate) != 0;
     static constexpr int one = kAcc ? 4 : 6, shared = kAcc ? 4 : 5;
-};
-template <int MODE> struct RingVmax<bf16, MODE> {
-    static constexpr int one = (MODE & kBwdRecompute) ? 3 : 4, shared = 3;
 };
 
 // Calls visitor.template ring<V, W>(); false when rows are wider than 4 warps

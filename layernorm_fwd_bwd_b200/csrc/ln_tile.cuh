@@ -157,7 +157,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const bool in = t + TPR * i < nvec;
-            to_pairs(xv[i], d[i]);
+            to_pairs<T>(xv[i], d[i]);
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 d[i][q] = sub2(d[i][q], K);
@@ -192,11 +192,11 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
             const int j = t + TPR * i;
             if (j < nvec) {
                 f32x2 wp[P], bp[P], o[P];
-                to_pairs(ws[j], wp);
-                to_pairs(bs[j], bp);
+                to_pairs<T>(ws[j], wp);
+                to_pairs<T>(bs[j], bp);
 #pragma unroll
                 for (int q = 0; q < P; ++q) o[q] = fma2(mul2(d[i][q], R), wp[q], bp[q]);
-                __stcs(yr + j, from_pairs(o));
+                __stcs(yr + j, from_pairs<T>(o));
             }
         }
         if (t == 0) {

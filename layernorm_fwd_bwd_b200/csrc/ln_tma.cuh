@@ -359,7 +359,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 for (int i = 0; i < V; ++i) {
                     const bool in = t + TPR * i < nvec;
                     f32x2 x[P];
-                    to_pairs(xv[i], x);
+                    to_pairs<T>(xv[i], x);
 #pragma unroll
                     for (int q = 0; q < P; ++q) {
                         const f32x2 dq = sub2(x[q], K);
@@ -378,7 +378,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 for (int i = 0; i < V; ++i) {
                     const bool in = t + TPR * i < nvec;
                     f32x2 x[P];
-                    if constexpr (!KEEP_D) to_pairs(xv[i], x);
+                    if constexpr (!KEEP_D) to_pairs<T>(xv[i], x);
 #pragma unroll
                     for (int q = 0; q < P; ++q) {
                         f32x2 dq;
@@ -407,13 +407,13 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 if constexpr (KEEP_D && !RECOMP) {
                     // d for every slot (dead lanes' values are never used)
                     f32x2 dq[P];
-                    to_pairs(xv[i], dq);
+                    to_pairs<T>(xv[i], dq);
 #pragma unroll
                     for (int q = 0; q < P; ++q) d[i][q] = sub2(dq[q], K);
                 }
                 if (j < nvec) {
                     f32x2 dy[P], wp[P];
-                    to_pairs(dv[i], dy);
+                    to_pairs<T>(dv[i], dy);
                     smem_pairs<P>(s_w + j * E, wp);
                     if constexpr (KEEP_G) {
 #pragma unroll
@@ -434,7 +434,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                         }
                     } else {
                         f32x2 x[P];
-                        to_pairs(xv[i], x);
+                        to_pairs<T>(xv[i], x);
 #pragma unroll
                         for (int q = 0; q < P; ++q) {
                             f32x2 dq = sub2(x[q], K);
@@ -486,11 +486,11 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                     }
                     if constexpr (ACC) {
                         f32x2 pp[P];
-                        to_pairs(ps[j], pp);
+                        to_pairs<T>(ps[j], pp);
 #pragma unroll
                         for (int q = 0; q < P; ++q) o[q] = add2(o[q], pp[q]);
                     }
-                    __stcs(gr + j, from_pairs(o));
+                    __stcs(gr + j, from_pairs<T>(o));
                 }
             }
             if constexpr (ACC) release();

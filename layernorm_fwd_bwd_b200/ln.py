@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(_PKG, "libln.so")
 
 LN_F32 = 0
 LN_BF16 = 1
+LN_F16 = 2
 
 LN_OK = 0
 LN_ERR_NULL = 1

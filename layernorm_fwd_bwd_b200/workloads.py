@@ -61,13 +61,13 @@ S_BRANCH, S_DINP_PREV, S_PARAM_PREV = 5, 6, 7
 
 EPS = float(np.float32(1e-5))
 
-F32, BF16 = "f32", "bf16"
+F32, BF16, F16 = "f32", "bf16", "f16"
 
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    dtype: str           # "f32" or "bf16": dtype of inp/out/dout/dinp/weight/bias
+    dtype: str           # "f32", "bf16" or "f16": dtype of inp/out/dout/dinp/weight/bias
     N: int               # rows (batch * sequence)
     C: int               # channels
     seed: int
@@ -155,9 +155,12 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def to_storage(v: np.ndarray, dtype: str) -> np.ndarray:
-    """float64 -> storage array (float32, or uint16 bf16 bit patterns)."""
+    """float64 -> storage array (float32, or uint16 bit patterns of bf16 /
+    fp16; numpy's float16 cast rounds to nearest-even)."""
     if dtype == F32:
         return np.asarray(v, dtype=np.float64).astype(np.float32)
+    if dtype == F16:
+        return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
     return round_bf16_bits(v)
 
 
@@ -165,12 +168,15 @@ def storage_to_f64(a: np.ndarray, dtype: str) -> np.ndarray:
     """Exact float64 values of a storage array."""
     if dtype == F32:
         return np.asarray(a, dtype=np.float32).astype(np.float64)
+    if dtype == F16:
+        return np.asarray(a, dtype=np.uint16).view(np.float16).astype(np.float64)
     return bf16_bits_to_f64(np.asarray(a, dtype=np.uint16))
 
 
 @dataclasses.dataclass
 class Batch:
-    """One batch of inputs in storage form (float32, or uint16 bf16 bits)."""
+    """One batch of inputs in storage form (float32, or uint16 bf16 / fp16
+    bits)."""
     workload: Workload
     rows: np.ndarray          # int64 row indices of the workload held here
     inp: np.ndarray           # [len(rows), C]

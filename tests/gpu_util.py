@@ -10,8 +10,8 @@ import torch
 
 from layernorm_fwd_bwd_b200 import workloads as wl
 
-DT = {"f32": 0, "bf16": 1}
-TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+DT = {"f32": 0, "bf16": 1, "f16": 2}
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
 def ln():
@@ -25,14 +25,21 @@ def to_device(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
     if dtype == "f32":
         return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
     bits = np.ascontiguousarray(a, np.uint16).view(np.int16)
-    return torch.from_numpy(bits).to(device).view(torch.bfloat16)
+    return torch.from_numpy(bits).to(device).view(TORCH_DT[dtype])
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
     t = t.detach().cpu()
     if t.dtype == torch.bfloat16:
         return wl.bf16_bits_to_f64(t.view(torch.int16).numpy().view(np.uint16))
+    if t.dtype == torch.float16:
+        return wl.storage_to_f64(t.view(torch.int16).numpy().view(np.uint16), "f16")
     return t.numpy().astype(np.float64)
+
+
+def bits(t: torch.Tensor) -> torch.Tensor:
+    """The tensor's bit patterns as integers (for bitwise comparisons)."""
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
 
 
 def nan_tensor(shape, tdtype, device="cuda") -> torch.Tensor:

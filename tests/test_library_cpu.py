@@ -60,7 +60,7 @@ def test_host_validation_without_gpu(lib):
     assert f(nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, None) == lib.LN_ERR_SHAPE
     assert f(nz, nz, nz, nz, nz, nz, 4, 0, 1e-5, 0, None) == lib.LN_ERR_SHAPE
     assert f(nz, nz, nz, nz, nz, nz, 4, (1 << 24) + 1, 1e-5, 0, None) == lib.LN_ERR_SHAPE
-    assert f(nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 2, None) == lib.LN_ERR_DTYPE
+    assert f(nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 3, None) == lib.LN_ERR_DTYPE
     assert f(nz, nz, nz, nz, nz, nz, 4, 8, 0.0, 0, None) == lib.LN_ERR_EPS
     assert f(nz, nz, nz, nz, nz, nz, 4, 8, float("nan"), 0, None) == lib.LN_ERR_EPS
     assert f(nz, nz, nz, nz, nz, nz, 4, 8, float("inf"), 1, None) == lib.LN_ERR_EPS
@@ -137,3 +137,9 @@ def test_tolerance_helpers():
     assert tol.rel_max(np.array([1e-3 + 1e-8]), np.array([1e-3]), scale=1.0) <= 1.1e-8
     with pytest.raises(AssertionError):
         tol.check("x", ref * (1 + 1e-4), ref, "f32", "act_fwd")
+    # one fp16 ulp at 1.0 is 2^-10; below 2^-14 the spacing stays 2^-24
+    assert tol.max_ulps(ref + np.array([2.0 ** -10, 0, 0]), ref, dtype="f16") == 1.0
+    assert tol.max_ulps(np.array([2.0 ** -24]), np.array([0.0]), dtype="f16") == 1.0
+    tol.check("x", ref + np.array([2.0 ** -9, 0, 0]), ref, "f16", "act_fwd")
+    with pytest.raises(AssertionError):
+        tol.check("x", ref + np.array([2.0 ** -8 * 1.01, 0, 0]), ref, "f16", "act_fwd")

@@ -100,7 +100,7 @@ SWEEP_C = [1, 2, 3, 7, 8, 31, 33, 127, 128, 768, 1023, 1024, 1600, 2048, 2056, 4
            8192, 16384, 20000]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", SWEEP_C)
 @pytest.mark.parametrize("N", [1, 3, 257])
 def test_shape_sweep(lib, dtype, C, N):
@@ -112,7 +112,7 @@ def test_shape_sweep(lib, dtype, C, N):
     _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", [768, 1600, 5])
 def test_misaligned_pointers(lib, dtype, C):
     """Arrays that start one element past a 16-byte boundary take the scalar
@@ -153,7 +153,7 @@ def test_misaligned_pointers(lib, dtype, C):
     tol.check("dbias", gu.to_f64(db), rb, dtype, "param_grad", sc["dbias"])
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", [768, 1600, 7, 20000])
 def test_guard_regions_and_full_coverage(lib, dtype, C):
     """Outputs sit inside larger buffers whose margins hold a sentinel; after
@@ -283,3 +283,20 @@ def test_repeated_runs_bitwise_identical(lib):
             for a, b in zip(first, cur):
                 assert torch.equal(a, b)
     assert lib.device_status() == 0
+
+
+def test_fp16_gpt2_124m_shape(lib):
+    """fp16 activations at the GPT-2 124M LayerNorm shape (65536 x 768,
+    the bf16 workload's distributions), every element: forward, backward as a
+    function of its arguments, and the forward feeding the backward."""
+    batch = wl.custom("f16", 65536, 768, seed=20240530, dout_sigma=0.02)
+    dev, (out, mean, rstd), ref_stats, res = _forward_parity(lib, batch, "f16 65536x768")
+    res += _backward_parity(lib, batch, dev, "f16 65536x768", ref_stats)
+    inp, wt, _, dout = dev
+    dinp, dw, db = gu.backward(lib, dout, inp, wt, mean, rstd, 65536, 768, "f16")
+    r = oracle.ln_backward(batch.f64("dout"), batch.f64("inp"), batch.f64("weight"),
+                           ref_stats[0], ref_stats[1])
+    res += [tol.check("f16 chained dinp", gu.to_f64(dinp), r[0], "f16", "act_bwd"),
+            tol.check("f16 chained dweight", gu.to_f64(dw), r[1], "f16", "param_grad"),
+            tol.check("f16 chained dbias", gu.to_f64(db), r[2], "f16", "param_grad")]
+    print(res)

@@ -28,7 +28,7 @@ def lib():
 
 
 def _fmt(dtype):
-    return "f32" if dtype == "f32" else "bf16"
+    return dtype          # the oracle's format names match the dtype names
 
 
 def _residual(lib, batch, extras, label, scaled=False):
@@ -56,8 +56,7 @@ def _residual(lib, batch, extras, label, scaled=False):
     # resid_out gives the same bits
     out2, mean2, rstd2 = gu.forward(lib, x, wt, bs, N, C, batch.eps, d)
     for a, b, n in ((out, out2, "out"), (mean, mean2, "mean"), (rstd, rstd2, "rstd")):
-        assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
-                           b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32)), \
+        assert torch.equal(gu.bits(a), gu.bits(b)), \
             f"{label}: fused {n} differs from ln_forward(resid_out)"
     return res
 
@@ -128,7 +127,7 @@ def test_backward_variants_full(lib, name, flags):
 SWEEP_C = [1, 3, 8, 33, 128, 512, 768, 1024, 1600, 2056, 3072, 4096, 20000]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", SWEEP_C)
 @pytest.mark.parametrize("N", [1, 257])
 def test_variant_sweep(lib, dtype, C, N):
@@ -143,7 +142,7 @@ def test_variant_sweep(lib, dtype, C, N):
         _backward_ex(lib, batch, extras, FLAG_SETS[fl], f"{label} {fl}", scaled=True)
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", [768, 1600, 5])
 def test_variants_misaligned(lib, dtype, C):
     """Arrays one element past a 16-byte boundary take the scalar kernels."""
@@ -239,3 +238,13 @@ def test_variant_edges(lib):
                        ACC_DINP | RECOMPUTE)
     torch.cuda.synchronize()
     assert torch.all(dinp == 7.0), "dinp of a one-column row is zero; 7 + 0 = 7"
+
+
+def test_fp16_variants_gpt2_124m_shape(lib):
+    """fp16 at the GPT-2 124M shape: the residual forward (sum bit-exact) and
+    the backward accumulating with recomputed statistics, every element."""
+    batch = wl.custom("f16", 65536, 768, seed=20240531, dout_sigma=0.02)
+    extras = wl.generate_extras(batch.workload)
+    res = _residual(lib, batch, extras, "f16 65536x768")
+    res += _backward_ex(lib, batch, extras, FLAG_SETS["acc_recompute"], "f16 65536x768 acc_rec")
+    print(res)

@@ -58,3 +58,14 @@ def test_compulsory_bytes():
     assert w.bwd_bytes() == 302_521_856
     assert wl.WORKLOADS["stress_fp32_65536x768"].fwd_bytes() + \
         wl.WORKLOADS["stress_fp32_65536x768"].bwd_bytes() == 1_007_696_896
+
+
+def test_f16_storage_roundtrip():
+    """fp16 storage holds numpy's nearest-even float16 of each draw, as 16-bit
+    patterns, and reads back exactly."""
+    b = wl.custom("f16", 8, 40, seed=9)
+    x = b.f64("inp")
+    assert b.inp.dtype == np.uint16
+    assert np.array_equal(x, b.inp.view(np.float16).astype(np.float64))
+    raw = wl._rows_block(b.workload, np.arange(8), wl.S_INP, 0.0, 1.0)
+    assert np.array_equal(x, raw.astype(np.float16).astype(np.float64))

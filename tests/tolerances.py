@@ -10,6 +10,11 @@ terms of ordinary size) from being judged in ulps of a tiny number; bf16 has
 8 significant bits, hence the 7.  mean, rstd, dweight and dbias stay fp32
 under bf16 activations: 1e-5 for mean/rstd, 1e-3 for dweight/dbias.
 
+fp16 tensors (no stated tolerance; the same rule carried over to fp16's 11
+significant bits): at most 2 fp16 ulps, 2^(floor(log2 m) - 10) at
+m = max(|v|, 2^-11 * max|ref|, 2^-14) (2^-14 is fp16's smallest normal, below
+which its spacing stays 2^-24); mean/rstd 1e-5, dweight/dbias 1e-3.
+
 These per-tensor rules are the stated ones for the five benchmark workloads.
 For other shapes (the sweep: single rows, C = 2, ...) a tensor's max-abs can
 be far below the size of the terms it is computed from: the mean of one
@@ -44,18 +49,26 @@ def rel_max(got, ref, scale: float = 0.0) -> float:
     return err / scale
 
 
-def bf16_ulp_error(got, ref, scale: float = 0.0) -> np.ndarray:
+# significant bits and smallest normal of the 16-bit formats
+_FMT = {"bf16": (8, 2.0 ** -126), "f16": (11, 2.0 ** -14)}
+
+
+def ulp_error(got, ref, scale: float = 0.0, dtype: str = "bf16") -> np.ndarray:
+    p, min_normal = _FMT[dtype]
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
-    floor = 2.0 ** -8 * max(float(np.max(np.abs(ref))) if ref.size else 0.0, scale)
-    m = np.maximum(np.abs(ref), floor)
-    m = np.where(m > 0, m, 2.0 ** -126)
-    ulp = np.exp2(np.floor(np.log2(m)) - 7)
+    floor = 2.0 ** -p * max(float(np.max(np.abs(ref))) if ref.size else 0.0, scale)
+    m = np.maximum(np.maximum(np.abs(ref), floor), min_normal)
+    ulp = np.exp2(np.floor(np.log2(m)) - (p - 1))
     return np.abs(got - ref) / ulp
 
 
-def max_ulps(got, ref, scale: float = 0.0) -> float:
-    e = bf16_ulp_error(got, ref, scale)
+def bf16_ulp_error(got, ref, scale: float = 0.0) -> np.ndarray:
+    return ulp_error(got, ref, scale, "bf16")
+
+
+def max_ulps(got, ref, scale: float = 0.0, dtype: str = "bf16") -> float:
+    e = ulp_error(got, ref, scale, dtype)
     return float(e.max()) if e.size else 0.0
 
 
@@ -78,9 +91,9 @@ def check(name: str, got, ref, dtype: str, kind: str, scale: float = 0.0) -> dic
     'param_grad' (dweight, dbias).  ``scale``: magnitude of the terms the
     result is computed from (0: the tensor's own max-abs alone).  Raises
     AssertionError past tolerance; returns the measured error."""
-    if kind in ("act_fwd", "act_bwd") and dtype == "bf16":
-        e = max_ulps(got, ref, scale)
-        assert e <= BF16_ULPS, f"{name}: {e:.3f} bf16 ulps > {BF16_ULPS}"
+    if kind in ("act_fwd", "act_bwd") and dtype in ("bf16", "f16"):
+        e = max_ulps(got, ref, scale, dtype)
+        assert e <= BF16_ULPS, f"{name}: {e:.3f} {dtype} ulps > {BF16_ULPS}"
         return {"name": name, "ulps": e}
     if dtype == "f32":
         tol = FP32_FWD if kind in ("act_fwd", "stats") else FP32_BWD
