@@ -3,9 +3,9 @@
 // chosen in exactly one place.
 //
 // Forward: rows of up to 8 vectors per lane take the one-shot tile kernel
-// (ln_tile.cuh): one warp per row up to 4 vectors, two warps per row for 5..8;
-// wider rows take the persistent register-resident kernel with W = 4, 8 or 16
-// warps per row and 4 vectors per thread.
+// (ln_tile.cuh) with one warp per row; wider rows take the persistent
+// register-resident kernel with W = 4, 8 or 16 warps per row and 4 vectors
+// per thread.
 // Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
 // persistent TMA-ring kernel (ln_tma.cuh) on one warp per row, wider rows the
 // ring with W = 2..4 warps per row; rows wider than that take the
@@ -45,11 +45,13 @@ constexpr int kTmaBwdConsumers = LN_TMA_BWD_CONSUMERS;
 template <int W> struct BwdRingConsumers {
     static constexpr int value = (kTmaBwdConsumers / W) * W;
 };
-// forward tile kernel: rows of up to 4 vectors per lane take one warp, wider
-// one-warp rows (5..8 vectors) are split over two warps (fewer registers,
-// more warps per SM)
+// forward tile kernel: one-warp rows of at least this many vectors per lane
+// are split over two warps.  Measured on B200 (bf16 C = 1600, 7 vectors per
+// lane): one warp 24.6-25.0 us, two warps of 4 vectors 25.6-27.0 us (a fifth
+// of their slots empty, plus two row exchanges); equal for fp32 C = 768.  So
+// rows up to 8 vectors stay on one warp (9: never split).
 #ifndef LN_TILE_FWD_W2_FROM_V
-#define LN_TILE_FWD_W2_FROM_V 5
+#define LN_TILE_FWD_W2_FROM_V 9
 #endif
 constexpr int kTileWarps = 8;                 // warps (= rows per tile) per tile block
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
@@ -117,8 +119,22 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
 // stages of the widest rows still fit in shared memory; recomputing the
 // statistics, bf16 rows of 4 vectors per lane would spill, so they go to two
 // warps.
+// 16-bit rows: the widest one-warp row and the vectors per lane when W > 1
+// warps share a row.  Measured on B200 (backward us, bf16): one = 4 / shared
+// = 3 gives C = 1024 41.7-43.0 and C = 1600 40.9-41.1; shared = 2 (C = 1600
+// on 4 warps, 78 % of the slots used against 69 %) 46.0-47.5 at C = 1600;
+// one = 3 with shared = 2 (C = 1024 on two warps, an exact fit) 46.5-49.1 at
+// C = 1024 -- the row exchanges cost more than the empty slots.
+#ifndef LN_RING_ONE_16
+#define LN_RING_ONE_16 4
+#endif
+#ifndef LN_RING_SHARED_16
+#define LN_RING_SHARED_16 3
+#endif
 template <typename T, int MODE> struct RingVmax {   // 16-bit elements (bf16, fp16)
-    static constexpr int one = (MODE & kBwdRecompute) ? 3 : 4, shared = 3;
+    static constexpr int one =
+        (MODE & kBwdRecompute) && LN_RING_ONE_16 > 3 ? 3 : LN_RING_ONE_16;
+    static constexpr int shared = LN_RING_SHARED_16;
 };
 template <int MODE> struct RingVmax<float, MODE> {
     static constexpr bool kAcc = (MODE & kBwdAccumulate) != 0;

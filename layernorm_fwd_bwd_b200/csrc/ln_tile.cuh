@@ -48,12 +48,18 @@ __device__ __forceinline__ bool tile_wait(uint64_t *bar, unsigned *status, unsig
 // vectors j = (w % W) * 32 + lane + i * 32 * W of it.  The pivot is the row's
 // first element, read from shared memory by every warp of the row; with
 // W > 1 the row sums meet through group_exchange (ln_tma.cuh).
+// Resident blocks per SM the register allocation must allow.  Wide 16-bit
+// rows (6+ vectors per lane, 2.4+ KB) fit three 2-tile blocks in shared memory;
+// unconstrained they take 82+ registers and only two blocks would fit.
+#ifndef LN_TILE_FWD_MINB
+#define LN_TILE_FWD_MINB(T, V) ((sizeof(T) == 2 && (V) >= 6) ? 3 : 0)
+#endif
 // Requirements (checked by the host): inp/out/weight/bias (and branch,
 // resid_out) 16-byte aligned, C * sizeof(T) a multiple of 16,
 // C / E <= 32 * W * V (== when FULL).
 // ---------------------------------------------------------------------------
 template <typename T, int V, int NW, int TILES, int W = 1, bool FULL = false, int MODE = 0>
-__global__ void __launch_bounds__(32 * NW)
+__global__ void __launch_bounds__(32 * NW, LN_TILE_FWD_MINB(T, V))
 ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                    const T *__restrict__ inp, const T *__restrict__ weight,
                    const T *__restrict__ bias, T *__restrict__ resid_out,
@@ -128,11 +134,15 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
         if (abort && W == 1) break;
         const unsigned char *row = s_tiles + (size_t(k) * RT + group) * row_bytes;
         const uint4 *src = reinterpret_cast<const uint4 *>(row);
+        // in(i, j): vector j of round i lies in the row.  With one warp per row
+        // the host picks V = ceil(nvec / 32), so rounds 0 .. V-2 are complete
+        // for every lane and only the last round needs the bound check.
+        auto in = [&](int i, int j) { return FULL || (W == 1 && i < V - 1) || j < nvec; };
         uint4 xv[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + TPR * i;
-            xv[i] = j < nvec ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+            xv[i] = in(i, j) ? src[j] : make_uint4(0u, 0u, 0u, 0u);
         }
         float pivot;
         if constexpr (RES) {
@@ -142,9 +152,9 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int j = t + TPR * i;
-                const uint4 bv = j < nvec ? src2[j] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 bv = in(i, j) ? src2[j] : make_uint4(0u, 0u, 0u, 0u);
                 xv[i] = add_round<T>(xv[i], bv);
-                if (j < nvec) __stcs(xo + j, xv[i]);
+                if (in(i, j)) __stcs(xo + j, xv[i]);
             }
             pivot = add_round1<T>(reinterpret_cast<const T *>(row)[0],
                                   reinterpret_cast<const T *>(row2)[0]);
@@ -156,12 +166,12 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
         f32x2 acc = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const bool in = t + TPR * i < nvec;
+            const bool live = in(i, t + TPR * i);
             to_pairs<T>(xv[i], d[i]);
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 d[i][q] = sub2(d[i][q], K);
-                if (in) acc = add2(acc, d[i][q]);
+                if (live) acc = add2(acc, d[i][q]);
             }
         }
         float sum = warp_sum(hsum(acc)), unused = 0.f;
@@ -173,11 +183,11 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
         f32x2 sq = pair(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const bool in = t + TPR * i < nvec;
+            const bool live = in(i, t + TPR * i);
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 d[i][q] = sub2(d[i][q], M);
-                if (in) sq = fma2(d[i][q], d[i][q], sq);
+                if (live) sq = fma2(d[i][q], d[i][q], sq);
             }
         }
         float var = warp_sum(hsum(sq));
@@ -190,7 +200,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int j = t + TPR * i;
-            if (j < nvec) {
+            if (in(i, j)) {
                 f32x2 wp[P], bp[P], o[P];
                 to_pairs<T>(ws[j], wp);
                 to_pairs<T>(bs[j], bp);
