@@ -194,6 +194,11 @@ __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, f
 // read at all but recomputed from the staged row (pivot x[r, 0], two-pass
 // deviations, as in the forward).
 // ---------------------------------------------------------------------------
+// Whether rows shared by W > 1 warps (plain backward) also keep g from pass 1.
+#ifndef LN_RING_KEEP_G_SHARED_PLAIN
+#define LN_RING_KEEP_G_SHARED_PLAIN 1
+#endif
+
 template <typename T, int V, int NC, int S, bool RR, int W = 1, int MODE = 0>
 __global__ void __launch_bounds__(32 * (NC + 1), (NC + 1) * 32 <= 256 ? 2 : 1)
 ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
@@ -347,7 +352,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             // that mean; from the saved statistics K = mean[r] and MD = 0.
             constexpr bool KEEP_D = sizeof(T) == 4 || V <= 3;
             constexpr bool KEEP_G =
-                KEEP_D && W == 1 && V <= (sizeof(T) == 4 ? (ACC ? 4 : 5) : (ACC ? 2 : 3));
+                KEEP_D && (W == 1 || LN_RING_KEEP_G_SHARED_PLAIN) &&
+                (W == 1 || MODE == 0) && V <= (sizeof(T) == 4 ? (ACC ? 4 : 5) : (ACC ? 2 : 3));
             uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
             f32x2 d[KEEP_D ? V : 1][P];
             f32x2 gk[KEEP_G ? V : 1][P];
