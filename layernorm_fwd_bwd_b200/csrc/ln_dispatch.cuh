@@ -27,6 +27,28 @@ namespace lnh {
 
 // ------------------------------------------------------------------ forward
 
+// Rows per one-shot block, at most `max_rows` and at least half of it: the
+// block count ceil(N / rows) is cut into ceil(blocks / resident) waves of
+// `resident` blocks, and a wave takes about as long as a block's rows, so
+// the value with the fewest rows in total (waves * rows) wins; ties go to
+// more rows per block.  GPT-2 1.5B (N = 16384, 444 resident): 13 rows, 3
+// full waves, instead of 16 rows and 2.3 waves.  Measured on B200: forward
+// 32.76 -> 32.29 us (124M), 22.94 -> 22.65 (350M), 21.02 -> 20.85 (1.5B);
+// less than the model says, since blocks of one wave do not end together.
+inline int tile_rows_per_block(int64_t N, int max_rows, int64_t resident) {
+    int best = max_rows;
+    int64_t best_cost = INT64_MAX;
+    for (int rows = max_rows; rows >= (max_rows + 1) / 2; --rows) {
+        const int64_t waves = ceil_div(ceil_div(N, rows), resident);
+        const int64_t cost = waves * rows;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = rows;
+        }
+    }
+    return best;
+}
+
 template <typename T, int MODE>
 struct FwdVec {
     const FwdArgs &a;
@@ -36,7 +58,7 @@ struct FwdVec {
     template <int V, int W, int GROUPS>
     void run() {
         if constexpr (W == 1) {
-            if (ceil_div(a.N, lnk::kTileWarps * lnk::kTileFwdTiles) <= INT32_MAX) {
+            if (ceil_div(a.N, lnk::kTileWarps) <= INT32_MAX) {
                 if constexpr (V >= LN_TILE_FWD_W2_FROM_V)
                     run_tile<(V + 1) / 2, 2>();
                 else
@@ -76,11 +98,13 @@ struct FwdVec {
         int occ = 0;
         err = blocks_per_sm(kern, a.dev, threads, smem, &occ);   // also sets the smem limit
         if (err != cudaSuccess) return;
-        const int64_t grid = ceil_div(a.N, (NW / RW) * TL);
+        const int rows = tile_rows_per_block(a.N, (NW / RW) * TL, int64_t(a.sms) * occ);
+        const int64_t grid = ceil_div(a.N, rows);
         err = launch(kern, (int)grid, threads, smem, a.stream, static_cast<T *>(a.out), a.mean,
                      a.rstd, static_cast<const T *>(a.inp), static_cast<const T *>(a.weight),
                      static_cast<const T *>(a.bias), static_cast<T *>(a.resid_out),
-                     static_cast<const T *>(a.branch), a.N, a.C, a.inv_C, a.eps, a.status);
+                     static_cast<const T *>(a.branch), a.N, a.C, a.inv_C, a.eps, rows,
+                     a.status);
     }
 };
 

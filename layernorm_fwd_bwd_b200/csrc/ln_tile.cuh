@@ -64,7 +64,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
                    const T *__restrict__ inp, const T *__restrict__ weight,
                    const T *__restrict__ bias, T *__restrict__ resid_out,
                    const T *__restrict__ branch, int64_t N, int C, float inv_C, float eps,
-                   unsigned *__restrict__ status) {
+                   int rows_pb, unsigned *__restrict__ status) {
     pdl_enter();
     constexpr bool RES = (MODE & kFwdResidual) != 0;
     constexpr int NS = RES ? 2 : 1;                           // input arrays
@@ -91,7 +91,10 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     const int group = warp / W;
     const int sub = warp - group * W;
     const int t = sub * 32 + lane;
-    const int64_t row0 = int64_t(blockIdx.x) * (RT * TILES);
+    // this block's rows: [row0, row_end), rows_pb <= RT * TILES of them (the
+    // host picks rows_pb so that the grid fills the resident blocks evenly)
+    const int64_t row0 = int64_t(blockIdx.x) * rows_pb;
+    const int64_t row_end = min64(N, row0 + rows_pb);
 
     if (threadIdx.x == 0) {
         for (int k = 0; k <= TILES; ++k) mbar_init(&bars[k], 1);
@@ -101,8 +104,8 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
         bulk_load(s_par + row_bytes, bias, row_bytes, &bars[0]);
         for (int k = 0; k < TILES; ++k) {
             const int64_t r = row0 + int64_t(k) * RT;
-            if (r < N) {
-                const uint32_t bytes = uint32_t(min64(RT, N - r)) * row_bytes;
+            if (r < row_end) {
+                const uint32_t bytes = uint32_t(min64(RT, row_end - r)) * row_bytes;
                 mbar_arrive_expect_tx(&bars[1 + k], NS * bytes);
                 bulk_load(s_tiles + size_t(k) * RT * row_bytes,
                           reinterpret_cast<const unsigned char *>(inp) + r * row_bytes, bytes,
@@ -129,7 +132,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     for (int k = 0; k < TILES; ++k) {
         if (abort && W == 1) break;
         const int64_t r = row0 + int64_t(k) * RT + group;
-        if (r >= N) break;                                    // uniform over the row group
+        if (r >= row_end) break;                              // uniform over the row group
         if (!tile_wait(&bars[1 + k], status, kStatusWaitFull)) abort = true;
         if (abort && W == 1) break;
         const unsigned char *row = s_tiles + (size_t(k) * RT + group) * row_bytes;
@@ -219,7 +222,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     // after a timeout, thread 0 waits (bounded) for every copy it issued.
     if (!__syncthreads_and(!abort) && threadIdx.x == 0) {
         for (int k = 0; k <= TILES; ++k) {
-            if (k > 0 && row0 + int64_t(k - 1) * RT >= N) break;
+            if (k > 0 && row0 + int64_t(k - 1) * RT >= row_end) break;
             if (!mbar_wait(&bars[k], 0)) atomicOr(status, kStatusDrain);
         }
     }

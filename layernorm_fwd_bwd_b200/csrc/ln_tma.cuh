@@ -343,7 +343,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             //   NC = -rstd^3*mean(g*d)   (xhat = d*rstd),
             // so pass 2 never unpacks x again; otherwise both passes rebuild
             // xhat from the packed row.  Where it also allows (KEEP_G: one warp
-            // per row, narrow enough rows), pass 1 keeps g = dout * weight too
+            // per row, or a shared row of the plain backward; narrow enough
+            // rows), pass 1 keeps g = dout * weight too
             // and adds the row's dout * xhat and dout to the column sums, so
             // pass 2 touches neither the packed dout nor the weight (the same
             // operations in the same order: identical results, about a fifth
