@@ -43,6 +43,10 @@
  *     a multiple of 16 bytes take the vectorised path; others a scalar path.
  *   - Errors are returned as an ln_status value; nothing is launched when
  *     validation fails, and no kernel asserts or traps.
+ *   - Calls can be captured into a CUDA graph (the backward's workspace then
+ *     becomes graph allocation nodes); make one uncaptured call of the same
+ *     shape on the device first, so that one-time set-up (the device's memory
+ *     pool, kernel attributes) happens outside the capture.
  *   - 1 <= C <= LN_MAX_C; 0 <= N <= LN_MAX_N; N * C <= LN_MAX_ELEMS.
  *     N == 0 launches nothing in the forward; in the backward it only
  *     zero-fills dweight and dbias (pointers other than dweight and dbias
