@@ -86,7 +86,9 @@ typedef enum {
     LN_ERR_WORKSPACE = 5,  /* the backward's workspace could not be allocated */
     LN_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
     LN_ERR_SCRATCH = 7,    /* ln_backward_noalloc: C > LN_NOALLOC_MAX_C */
-    LN_ERR_FLAGS = 8       /* ln_backward_ex: unknown bits in flags */
+    LN_ERR_FLAGS = 8,      /* ln_backward_ex: unknown bits in flags */
+    LN_ERR_ALIAS = 9       /* an output overlaps an input (or another output)
+                              where this header forbids it */
 } ln_status;
 
 /*
@@ -97,7 +99,8 @@ typedef enum {
  *   inp   [N*C] dtype, read
  *   weight, bias [C] dtype, read
  *   eps   finite, > 0 (1e-5 in GPT-2)
- * out must not overlap inp.  Returns LN_OK or an ln_status error.
+ * out must not overlap inp (LN_ERR_ALIAS).  Returns LN_OK or an ln_status
+ * error.
  */
 int ln_forward(void *out, float *mean, float *rstd, const void *inp,
                const void *weight, const void *bias, int64_t N, int64_t C,
@@ -117,8 +120,8 @@ int ln_forward(void *out, float *mean, float *rstd, const void *inp,
  * per-block partial sums into a library-owned workspace drawn, stream-ordered,
  * from a per-device memory pool (returned to the pool on `stream` after use),
  * then one fixed-order sum of the partials.  dinp must not overlap dout or
- * inp.  Returns LN_OK or an ln_status error (LN_ERR_WORKSPACE when the pool
- * cannot supply the workspace).
+ * inp (LN_ERR_ALIAS).  Returns LN_OK or an ln_status error (LN_ERR_WORKSPACE
+ * when the pool cannot supply the workspace).
  */
 int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
                 const void *inp, const void *weight, const float *mean,
@@ -142,7 +145,7 @@ int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
  *   resid, branch [N*C] dtype, read      the two summands
  *   weight, bias [C] dtype, read; eps as in ln_forward
  * resid_out and out must not overlap each other or any input (no in-place
- * update).  Bytes moved: 4*N*C*size (two reads, two writes) against 5*N*C*size
+ * update; LN_ERR_ALIAS).  Bytes moved: 4*N*C*size (two reads, two writes) against 5*N*C*size
  * for a separate add and ln_forward.  Returns LN_OK or an ln_status error.
  */
 int ln_forward_residual(void *resid_out, void *out, float *mean, float *rstd,

@@ -90,6 +90,13 @@ int check_shape(int64_t N, int64_t C) {
 }
 
 bool valid_dtype(int dtype) { return dtype == LN_F32 || dtype == LN_BF16 || dtype == LN_F16; }
+size_t elem_size(int dtype) { return dtype == LN_F32 ? 4 : 2; }
+
+// Whether the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
 bool valid_eps(float eps) { return std::isfinite(eps) && eps > 0.f; }
 
 template <typename T>
@@ -117,6 +124,11 @@ int forward_entry(void *out, float *mean, float *rstd, const void *inp, const vo
     if (N == 0) return LN_OK;
     if (!out || !mean || !rstd || !inp || !weight || !bias) return LN_ERR_NULL;
     if (residual && (!resid_out || !branch)) return LN_ERR_NULL;
+    const size_t act = size_t(N) * size_t(C) * elem_size(dtype);
+    if (overlap(out, act, inp, act)) return LN_ERR_ALIAS;
+    if (residual && (overlap(out, act, branch, act) || overlap(resid_out, act, inp, act) ||
+                     overlap(resid_out, act, branch, act) || overlap(resid_out, act, out, act)))
+        return LN_ERR_ALIAS;
     int dev = 0;
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
@@ -174,6 +186,8 @@ int backward_entry(void *dinp, float *dweight, float *dbias, const void *dout,
     }
     if (!dinp || !dout || !inp || !weight) return LN_ERR_NULL;
     if (!recompute && (!mean || !rstd)) return LN_ERR_NULL;
+    const size_t act = size_t(N) * size_t(C) * elem_size(dtype);
+    if (overlap(dinp, act, dout, act) || overlap(dinp, act, inp, act)) return LN_ERR_ALIAS;
     int dev = 0;
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
@@ -235,6 +249,7 @@ const char *ln_status_string(int status) {
         case LN_ERR_CUDA: return "LN_ERR_CUDA: a CUDA runtime call or kernel launch failed";
         case LN_ERR_SCRATCH: return "LN_ERR_SCRATCH: C exceeds the static scratch of ln_backward_noalloc";
         case LN_ERR_FLAGS: return "LN_ERR_FLAGS: unknown bits in the flags of ln_backward_ex";
+        case LN_ERR_ALIAS: return "LN_ERR_ALIAS: an output overlaps an input or another output";
         default: return "unknown ln_status";
     }
 }

@@ -30,6 +30,7 @@ LN_ERR_WORKSPACE = 5
 LN_ERR_CUDA = 6
 LN_ERR_SCRATCH = 7
 LN_ERR_FLAGS = 8
+LN_ERR_ALIAS = 9
 LN_BWD_ACCUMULATE_DINP = 1
 LN_BWD_ACCUMULATE_DPARAMS = 2
 LN_BWD_RECOMPUTE_STATS = 4

@@ -45,7 +45,8 @@ def test_exports_every_declared_symbol(lib):
 
 def test_status_strings(lib):
     names = ["LN_OK", "LN_ERR_NULL", "LN_ERR_SHAPE", "LN_ERR_DTYPE", "LN_ERR_EPS",
-             "LN_ERR_WORKSPACE", "LN_ERR_CUDA", "LN_ERR_SCRATCH", "LN_ERR_FLAGS"]
+             "LN_ERR_WORKSPACE", "LN_ERR_CUDA", "LN_ERR_SCRATCH", "LN_ERR_FLAGS",
+             "LN_ERR_ALIAS"]
     for code, name in enumerate(names):
         assert lib.ln_status_string(code).startswith(name)
         assert getattr(lib, name) == code
@@ -106,6 +107,30 @@ def test_variant_validation_without_gpu(lib):
     # N == 0 with accumulated parameters has nothing to do (no memset either)
     assert x(None, nz, nz, None, None, None, None, None, 0, 8, 0.0, 0,
              lib.LN_BWD_ACCUMULATE_DPARAMS, None) == lib.LN_OK
+    assert lib.launch_count() == 0
+
+
+def test_overlapping_outputs_are_refused_without_gpu(lib):
+    """Outputs that overlap inputs where the header forbids it return
+    LN_ERR_ALIAS before any CUDA call (addresses are never dereferenced; every
+    case here is refused on the host, so none can reach a device)."""
+    N, C = 4, 8
+    act = N * C * 2                      # bytes of one bf16 activation array
+    a, b, c, d = 1 << 20, 2 << 20, 3 << 20, 4 << 20   # disjoint fake device addresses
+    f = lib.raw_forward
+    assert f(a, b, b + 64, a, c, d, N, C, 1e-5, 1, None) == lib.LN_ERR_ALIAS       # out == inp
+    assert f(a, b, b + 64, a + act - 2, c, d, N, C, 1e-5, 1, None) == lib.LN_ERR_ALIAS
+    r = lib.raw_forward_residual
+    assert r(a, b, c, c + 64, a, d, c + 128, c + 256, N, C, 1e-5, 1, None) == lib.LN_ERR_ALIAS
+    assert r(a, b, c, c + 64, d, b + 2, c + 128, c + 256, N, C, 1e-5, 1, None) == lib.LN_ERR_ALIAS
+    assert r(a, a + 16, c, c + 64, d, d + act, c + 128, c + 256, N, C, 1e-5, 1,
+             None) == lib.LN_ERR_ALIAS                                               # outputs
+    bw = lib.raw_backward
+    assert bw(a, c, c + 64, a, b, d, c + 128, c + 256, N, C, 1, None) == lib.LN_ERR_ALIAS
+    assert bw(a, c, c + 64, b, a + 8, d, c + 128, c + 256, N, C, 1, None) == lib.LN_ERR_ALIAS
+    x = lib.raw_backward_ex
+    assert x(a, c, c + 64, a, b, d, None, None, N, C, 1e-5, 1, lib.LN_BWD_RECOMPUTE_STATS,
+             None) == lib.LN_ERR_ALIAS
     assert lib.launch_count() == 0
 
 

@@ -350,3 +350,25 @@ def test_cuda_graph_capture_replays_bitwise(lib):
         for k, v in o.items():
             assert torch.equal(gu.bits(v), eager[k]), f"graph replay: {k} differs"
     assert lib.device_status() == 0
+
+
+def test_aliased_outputs_refused(lib):
+    """In-place calls the header forbids raise LN_ERR_ALIAS and launch
+    nothing: out == inp, dinp == dout, resid_out == resid."""
+    N, C = 64, 768
+    x = torch.randn(N, C, device="cuda").to(torch.bfloat16)
+    w = torch.ones(C, device="cuda", dtype=torch.bfloat16)
+    m = torch.empty(N, device="cuda")
+    r = torch.empty(N, device="cuda")
+    dw = torch.empty(C, device="cuda")
+    n0 = lib.launch_count()
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_forward(x, m, r, x, w, w, N, C, 1e-5, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_backward(x, dw, dw.clone(), x, x.clone(), w, m, r, N, C, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_forward_residual(x, x.clone(), m, r, x, x.clone(), w, w, N, C, 1e-5, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    assert lib.launch_count() == n0
