@@ -80,11 +80,38 @@ def parse_args():
     return p.parse_args()
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments (string and character literals kept
+    intact), each line's trailing blanks and blank lines dropped, so that
+    editing a comment does not change the hash of the code."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            end = src.find("*/", i + 2)
+            i = n if end < 0 else end + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [line.rstrip() for line in "".join(out).split("\n")]
+    return "\n".join(line for line in lines if line)
+
+
 def source_sha256() -> str:
+    """Hash of the kernel sources' code (comments excluded)."""
     h = hashlib.sha256()
     for path in KERNEL_SOURCES:
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -1,6 +1,8 @@
-// ln_tma.cuh -- LayerNorm forward and backward fed by a TMA bulk-copy ring.
+// ln_tma.cuh -- the TMA and mbarrier helpers (bounded waits, 1-D bulk copies,
+// also used by the one-shot forward in ln_tile.cuh) and the LayerNorm
+// backward fed by a TMA bulk-copy ring.
 //
-// Why: the register-resident kernels keep at most one row per warp in flight
+// Why a ring: the register-resident kernels keep at most one row per warp in flight
 // (1.5 KB for a bf16 row of 768), and a warp spends most of each row on
 // arithmetic, so a bf16 launch cannot keep enough bytes in flight to reach
 // the HBM roofline.  Here one producer warp per block streams whole tiles of
