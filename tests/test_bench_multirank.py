@@ -63,3 +63,15 @@ def test_reference_arm_runs_on_rank_zero_only():
     line = bench.run_reference(args, world=1, rank=0)
     assert line["impl"] == "reference" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["unit"] == "GB/s" and line["value"] > 0
+
+
+def test_source_hash_ignores_comments_only():
+    """The traffic figure's key: comment edits keep it, code edits change it,
+    and string literals (inline PTX) survive comment stripping."""
+    a = 'asm("mov.u32 %0, 1; // not a comment");  // comment\nint x = 2; /* c */\n'
+    b = 'asm("mov.u32 %0, 1; // not a comment");  // other words\n\nint x = 2;\n'
+    c = 'asm("mov.u32 %0, 1; // not a comment");\nint x = 3;\n'
+    assert bench.strip_comments(a) == bench.strip_comments(b)
+    assert bench.strip_comments(a) != bench.strip_comments(c)
+    assert "// not a comment" in bench.strip_comments(a)
+    assert len(bench.source_sha256()) == 64
