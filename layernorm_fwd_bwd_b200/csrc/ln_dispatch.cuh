@@ -78,20 +78,38 @@ struct FwdVec {
                      static_cast<const T *>(a.bias), static_cast<T *>(a.resid_out),
                      static_cast<const T *>(a.branch), a.N, a.C, a.inv_C, a.eps);
     }
+    // Rows of 9..16 vectors per lane on two warps per row (V per warp).  When
+    // two tiles per block do not fit in shared memory (the residual
+    // variant's two arrays at bf16 C > 3.4K), one tile per block: a row's
+    // arithmetic does not depend on the tile count, so the residual forward
+    // still normalises exactly as ln_forward of its stored sum would.
+    template <int V>
+    void run_tile_two() {
+        constexpr int NW = lnk::kTileWarps * 2;
+        constexpr int TL = lnk::kTileFwdTiles;
+        if (ceil_div(a.N, lnk::kTileWarps) > INT32_MAX) {
+            run<4, 4, 2>();
+        } else if (lnk::fwd_tile_smem<T, NW, TL, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+            run_tile<V, 2>();
+        } else if (lnk::fwd_tile_smem<T, NW, 1, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+            run_tile<V, 2, 1>();
+        } else {
+            run<4, 4, 2>();
+        }
+    }
     // Rows that fill every lane's V vectors exactly take a variant without
     // per-vector bound checks.
-    template <int V, int RW>
+    template <int V, int RW, int TL = lnk::kTileFwdTiles>
     void run_tile() {
         constexpr int E = lnk::Vec<T>::E;
         if (a.C / E == 32 * RW * V)
-            run_tile_k<V, RW, true>();
+            run_tile_k<V, RW, TL, true>();
         else
-            run_tile_k<V, RW, false>();
+            run_tile_k<V, RW, TL, false>();
     }
-    template <int V, int RW, bool FULL>
+    template <int V, int RW, int TL, bool FULL>
     void run_tile_k() {
         constexpr int NW = lnk::kTileWarps * RW;          // 8 rows per tile either way
-        constexpr int TL = lnk::kTileFwdTiles;
         auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL, RW, FULL, MODE>;
         const int threads = 32 * NW;
         const size_t smem = lnk::fwd_tile_smem<T, NW, TL, RW, kArrays>(a.C);

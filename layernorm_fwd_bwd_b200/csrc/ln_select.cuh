@@ -53,6 +53,12 @@ template <int W> struct BwdRingConsumers {
 #ifndef LN_TILE_FWD_W2_FROM_V
 #define LN_TILE_FWD_W2_FROM_V 9
 #endif
+// Rows of 9..16 vectors per lane (bf16 C = 2049..4096): the tile kernel with
+// two warps per row (at most 8 vectors per lane each) instead of the
+// register-resident kernel with four.
+#ifndef LN_TILE_FWD_TWO_WARPS
+#define LN_TILE_FWD_TWO_WARPS 1
+#endif
 constexpr int kTileWarps = 8;                 // warps (= rows per tile) per tile block
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
 
@@ -101,6 +107,15 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
         case 7: v.template run<7, 1, LN_FWD_GROUPS_W1>(); return true;
         case 8: v.template run<8, 1, LN_FWD_GROUPS_W1>(); return true;
         default: break;
+    }
+    if constexpr (LN_TILE_FWD_TWO_WARPS) {
+        switch ((nvec + 63) / 64) {          // vectors per lane on two warps per row
+            case 5: v.template run_tile_two<5>(); return true;
+            case 6: v.template run_tile_two<6>(); return true;
+            case 7: v.template run_tile_two<7>(); return true;
+            case 8: v.template run_tile_two<8>(); return true;
+            default: break;
+        }
     }
     if (nvec <= 4 * 32 * 4) { v.template run<4, 4, 2>(); return true; }
     if (nvec <= 8 * 32 * 4) { v.template run<4, 8, 1>(); return true; }

@@ -49,17 +49,18 @@ __device__ __forceinline__ bool tile_wait(uint64_t *bar, unsigned *status, unsig
 // first element, read from shared memory by every warp of the row; with
 // W > 1 the row sums meet through group_exchange (ln_tma.cuh).
 // Resident blocks per SM the register allocation must allow.  Wide 16-bit
-// rows (6+ vectors per lane, 2.4+ KB) fit three 2-tile blocks in shared memory;
-// unconstrained they take 82+ registers and only two blocks would fit.
+// rows on one warp (6+ vectors per lane, 2.4+ KB) fit three 2-tile blocks of
+// 8 warps in shared memory; unconstrained they take 82+ registers and only
+// two blocks would fit.  (0: no constraint.)
 #ifndef LN_TILE_FWD_MINB
-#define LN_TILE_FWD_MINB(T, V) ((sizeof(T) == 2 && (V) >= 6) ? 3 : 0)
+#define LN_TILE_FWD_MINB(T, V, NW) (((NW) == 8 && sizeof(T) == 2 && (V) >= 6) ? 3 : 0)
 #endif
 // Requirements (checked by the host): inp/out/weight/bias (and branch,
 // resid_out) 16-byte aligned, C * sizeof(T) a multiple of 16,
 // C / E <= 32 * W * V (== when FULL).
 // ---------------------------------------------------------------------------
 template <typename T, int V, int NW, int TILES, int W = 1, bool FULL = false, int MODE = 0>
-__global__ void __launch_bounds__(32 * NW, LN_TILE_FWD_MINB(T, V))
+__global__ void __launch_bounds__(32 * NW, LN_TILE_FWD_MINB(T, V, NW))
 ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restrict__ rstd,
                    const T *__restrict__ inp, const T *__restrict__ weight,
                    const T *__restrict__ bias, T *__restrict__ resid_out,
