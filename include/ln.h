@@ -39,6 +39,11 @@
  *     ln_backward_ex is asked to accumulate.
  *   - Results are deterministic: the same inputs give bitwise-identical
  *     outputs on every call (no floating-point atomics).
+ *   - No call works in place: an output must not share a byte with another
+ *     output or with an array the call reads (LN_ERR_ALIAS, checked on the
+ *     host before anything is launched).  Inputs may overlap one another.
+ *     The accumulating backward reads the outputs it adds to; that is the
+ *     same array, not an overlap.
  *   - Any alignment is accepted.  Fully 16-byte-aligned arrays with C * size
  *     a multiple of 16 bytes take the vectorised path; others a scalar path.
  *   - Errors are returned as an ln_status value; nothing is launched when
@@ -87,8 +92,8 @@ typedef enum {
     LN_ERR_CUDA = 6,       /* a CUDA runtime call or launch failed */
     LN_ERR_SCRATCH = 7,    /* ln_backward_noalloc: C > LN_NOALLOC_MAX_C */
     LN_ERR_FLAGS = 8,      /* ln_backward_ex: unknown bits in flags */
-    LN_ERR_ALIAS = 9       /* an output overlaps an input (or another output)
-                              where this header forbids it */
+    LN_ERR_ALIAS = 9       /* an output overlaps another output or an array
+                              the call reads */
 } ln_status;
 
 /*
@@ -99,8 +104,8 @@ typedef enum {
  *   inp   [N*C] dtype, read
  *   weight, bias [C] dtype, read
  *   eps   finite, > 0 (1e-5 in GPT-2)
- * out must not overlap inp (LN_ERR_ALIAS).  Returns LN_OK or an ln_status
- * error.
+ * out, mean and rstd must not overlap one another or inp, weight or bias
+ * (LN_ERR_ALIAS).  Returns LN_OK or an ln_status error.
  */
 int ln_forward(void *out, float *mean, float *rstd, const void *inp,
                const void *weight, const void *bias, int64_t N, int64_t C,
@@ -119,9 +124,10 @@ int ln_forward(void *out, float *mean, float *rstd, const void *inp,
  * The column sums are formed in two stages with a fixed summation order:
  * per-block partial sums into a library-owned workspace drawn, stream-ordered,
  * from a per-device memory pool (returned to the pool on `stream` after use),
- * then one fixed-order sum of the partials.  dinp must not overlap dout or
- * inp (LN_ERR_ALIAS).  Returns LN_OK or an ln_status error (LN_ERR_WORKSPACE
- * when the pool cannot supply the workspace).
+ * then one fixed-order sum of the partials.  dinp, dweight and dbias must
+ * not overlap one another or dout, inp, weight, mean or rstd (LN_ERR_ALIAS).
+ * Returns LN_OK or an ln_status error (LN_ERR_WORKSPACE when the pool cannot
+ * supply the workspace).
  */
 int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
                 const void *inp, const void *weight, const float *mean,
@@ -144,8 +150,8 @@ int ln_backward(void *dinp, float *dweight, float *dbias, const void *dout,
  *   out, mean, rstd                      as in ln_forward
  *   resid, branch [N*C] dtype, read      the two summands
  *   weight, bias [C] dtype, read; eps as in ln_forward
- * resid_out and out must not overlap each other or any input (no in-place
- * update; LN_ERR_ALIAS).  Bytes moved: 4*N*C*size (two reads, two writes) against 5*N*C*size
+ * resid_out, out, mean and rstd must not overlap one another or any input
+ * (no in-place update; LN_ERR_ALIAS).  Bytes moved: 4*N*C*size (two reads, two writes) against 5*N*C*size
  * for a separate add and ln_forward.  Returns LN_OK or an ln_status error.
  */
 int ln_forward_residual(void *resid_out, void *out, float *mean, float *rstd,
@@ -178,8 +184,9 @@ int ln_forward_residual(void *resid_out, void *out, float *mean, float *rstd,
  *          and LN_BWD_RECOMPUTE_STATS; other bits give LN_ERR_FLAGS
  * With LN_BWD_ACCUMULATE_DINP, dinp is read as well as written (it must hold
  * the previous gradient); with LN_BWD_ACCUMULATE_DPARAMS, dweight and dbias
- * are read and N == 0 leaves them unchanged.  The column sums keep their
- * fixed order, so results stay deterministic.
+ * are read and N == 0 leaves them unchanged.  With LN_BWD_RECOMPUTE_STATS
+ * mean and rstd are not read, so their overlaps are not checked.  The column
+ * sums keep their fixed order, so results stay deterministic.
  */
 int ln_backward_ex(void *dinp, float *dweight, float *dbias, const void *dout,
                    const void *inp, const void *weight, const float *mean,

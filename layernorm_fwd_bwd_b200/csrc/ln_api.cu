@@ -97,6 +97,22 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return na && nb && x < y + nb && y < x + na;
 }
+
+// One array of a call: its address and size in bytes (0 for an array the
+// call does not touch).
+struct Span {
+    const void *p;
+    size_t n;
+};
+
+// Whether one of the first n_out spans (the call's outputs) shares a byte
+// with any other span of the call.
+bool aliased(const Span *s, int n_out, int n) {
+    for (int i = 0; i < n_out; ++i)
+        for (int j = 0; j < n; ++j)
+            if (j != i && overlap(s[i].p, s[i].n, s[j].p, s[j].n)) return true;
+    return false;
+}
 bool valid_eps(float eps) { return std::isfinite(eps) && eps > 0.f; }
 
 template <typename T>
@@ -125,10 +141,11 @@ int forward_entry(void *out, float *mean, float *rstd, const void *inp, const vo
     if (!out || !mean || !rstd || !inp || !weight || !bias) return LN_ERR_NULL;
     if (residual && (!resid_out || !branch)) return LN_ERR_NULL;
     const size_t act = size_t(N) * size_t(C) * elem_size(dtype);
-    if (overlap(out, act, inp, act)) return LN_ERR_ALIAS;
-    if (residual && (overlap(out, act, branch, act) || overlap(resid_out, act, inp, act) ||
-                     overlap(resid_out, act, branch, act) || overlap(resid_out, act, out, act)))
-        return LN_ERR_ALIAS;
+    const size_t par = size_t(C) * elem_size(dtype), stat = size_t(N) * sizeof(float);
+    const size_t racts = residual ? act : 0;
+    const Span spans[] = {{out, act},  {mean, stat},   {rstd, stat}, {resid_out, racts},
+                          {inp, act},  {weight, par},  {bias, par},  {branch, racts}};
+    if (aliased(spans, 4, 8)) return LN_ERR_ALIAS;
     int dev = 0;
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
@@ -187,7 +204,11 @@ int backward_entry(void *dinp, float *dweight, float *dbias, const void *dout,
     if (!dinp || !dout || !inp || !weight) return LN_ERR_NULL;
     if (!recompute && (!mean || !rstd)) return LN_ERR_NULL;
     const size_t act = size_t(N) * size_t(C) * elem_size(dtype);
-    if (overlap(dinp, act, dout, act) || overlap(dinp, act, inp, act)) return LN_ERR_ALIAS;
+    const size_t par = size_t(C) * elem_size(dtype), grad = size_t(C) * sizeof(float);
+    const size_t stat = recompute ? 0 : size_t(N) * sizeof(float);   // unread when recomputed
+    const Span spans[] = {{dinp, act}, {dweight, grad}, {dbias, grad}, {dout, act},
+                          {inp, act},  {weight, par},   {mean, stat},  {rstd, stat}};
+    if (aliased(spans, 3, 8)) return LN_ERR_ALIAS;
     int dev = 0;
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;

@@ -134,6 +134,79 @@ def test_overlapping_outputs_are_refused_without_gpu(lib):
     assert lib.launch_count() == 0
 
 
+def test_every_output_overlap_is_refused_without_gpu(lib):
+    """No output may share a byte with another output or with any array the
+    call reads: the statistics, the parameter gradients and the small arrays
+    included.  Each case starts from a layout of disjoint fake addresses and
+    moves one array onto another; all are refused on the host."""
+    N, C = 4, 8
+    act, par, stat, grad = N * C * 2, C * 2, N * 4, C * 4     # bf16 sizes in bytes
+    base = 1 << 20
+    fwd = dict(out=base, mean=2 * base, rstd=3 * base, inp=4 * base, weight=5 * base,
+               bias=6 * base)
+
+    def f(**moved):
+        p = {**fwd, **moved}
+        return lib.raw_forward(p["out"], p["mean"], p["rstd"], p["inp"], p["weight"],
+                               p["bias"], N, C, 1e-5, 1, None)
+
+    for moved in (dict(rstd=fwd["mean"]),                    # mean == rstd
+                  dict(rstd=fwd["mean"] + stat - 4),         # last float shared
+                  dict(mean=fwd["out"] + act - 4),           # mean inside out's tail
+                  dict(out=fwd["rstd"] + 4),                 # out over rstd
+                  dict(mean=fwd["weight"] + par - 2),        # mean over weight's last element
+                  dict(rstd=fwd["bias"]),
+                  dict(mean=fwd["inp"] + 2 * C)):
+        assert f(**moved) == lib.LN_ERR_ALIAS, moved
+
+    res = dict(fwd, resid_out=7 * base, branch=8 * base)
+
+    def r(**moved):
+        p = {**res, **moved}
+        return lib.raw_forward_residual(p["resid_out"], p["out"], p["mean"], p["rstd"],
+                                        p["inp"], p["branch"], p["weight"], p["bias"], N, C,
+                                        1e-5, 1, None)
+
+    for moved in (dict(mean=res["resid_out"] + 8), dict(resid_out=res["weight"]),
+                  dict(rstd=res["branch"] + act - 4), dict(out=res["branch"])):
+        assert r(**moved) == lib.LN_ERR_ALIAS, moved
+
+    bwd = dict(dinp=base, dweight=2 * base, dbias=3 * base, dout=4 * base, inp=5 * base,
+               weight=6 * base, mean=7 * base, rstd=8 * base)
+
+    def b(flags=0, **moved):
+        p = {**bwd, **moved}
+        return lib.raw_backward_ex(p["dinp"], p["dweight"], p["dbias"], p["dout"], p["inp"],
+                                   p["weight"], p["mean"], p["rstd"], N, C, 1e-5, 1, flags,
+                                   None)
+
+    acc = lib.LN_BWD_ACCUMULATE_DINP | lib.LN_BWD_ACCUMULATE_DPARAMS
+    for flags in (0, acc):
+        for moved in (dict(dbias=bwd["dweight"]),                 # dweight == dbias
+                      dict(dbias=bwd["dweight"] + grad - 4),
+                      dict(dweight=bwd["weight"]),                # dweight over weight
+                      dict(dbias=bwd["mean"] + stat - 4),         # dbias over mean's tail
+                      dict(dweight=bwd["rstd"]),
+                      dict(dweight=bwd["inp"] + act - 4),
+                      dict(dbias=bwd["dinp"] + 16),               # over another output
+                      dict(dinp=bwd["weight"] - act + 2)):        # dinp's tail over weight
+            assert b(flags, **moved) == lib.LN_ERR_ALIAS, (flags, moved)
+    # the plain and no-alloc entry points share the checks
+    p = dict(bwd, dbias=bwd["dweight"])
+    assert lib.raw_backward(p["dinp"], p["dweight"], p["dbias"], p["dout"], p["inp"],
+                            p["weight"], p["mean"], p["rstd"], N, C, 1, None) == lib.LN_ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        # without a device the no-alloc call stops at its device lookup,
+        # before the shared checks; with one it reaches them
+        pytest.skip("ln_backward_noalloc reaches the shared checks only with a device")
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_backward_noalloc(p["dinp"], p["dweight"], p["dbias"], p["dout"], p["inp"],
+                                p["weight"], p["mean"], p["rstd"], N, C, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    assert lib.launch_count() == 0
+
+
 def test_binding_raises_lnerror(lib):
     with pytest.raises(lib.LNError) as e:
         lib.ln_forward(16, 16, 16, 16, 16, 16, -3, 8, 1e-5, 0, stream=0)
