@@ -3,8 +3,9 @@
 // instantiates these once per combination (each in its own object, so the
 // kernels of the combinations compile in parallel).
 //
-// Geometry.  The forward's tile kernel runs one block per 16 rows (one-shot);
-// every other kernel runs on a persistent grid of (SM count) x (resident
+// Geometry.  The forward's tile kernel runs one block per 8 to 16 rows
+// (one-shot; tile_rows_per_block picks the count); every other kernel runs on
+// a persistent grid of (SM count) x (resident
 // blocks per SM, from the occupancy calculator for the exact block size and
 // shared memory), capped by the number of rows.  Arrays that are all 16-byte
 // aligned, with C * sizeof(T) a multiple of 16, take the vectorised kernels

@@ -3,9 +3,9 @@
 // chosen in exactly one place.
 //
 // Forward: rows of up to 8 vectors per lane take the one-shot tile kernel
-// (ln_tile.cuh) with one warp per row; wider rows take the persistent
-// register-resident kernel with W = 4, 8 or 16 warps per row and 4 vectors
-// per thread.
+// (ln_tile.cuh) with one warp per row, rows of 9..16 the same kernel with two
+// warps per row; wider rows take the persistent register-resident kernel
+// with W = 4, 8 or 16 warps per row and 4 vectors per thread.
 // Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
 // persistent TMA-ring kernel (ln_tma.cuh) on one warp per row, wider rows the
 // ring with W = 2..4 warps per row; rows wider than that take the
@@ -59,7 +59,7 @@ template <int W> struct BwdRingConsumers {
 #ifndef LN_TILE_FWD_TWO_WARPS
 #define LN_TILE_FWD_TWO_WARPS 1
 #endif
-constexpr int kTileWarps = 8;                 // warps (= rows per tile) per tile block
+constexpr int kTileWarps = 8;   // rows per forward tile (warps per tile, doubled at two per row)
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
 
 // Arrays streamed through the backward ring: inp and dout, plus the previous
