@@ -10,12 +10,19 @@ machine where the CUDA library has not been built; calling any entry point
 without the library raises immediately (there is no CPU fallback).
 """
 
-_BINDING_NAMES = ("ln_forward", "ln_backward", "ln_status_string", "LNError",
-                  "LN_F32", "LN_BF16", "library_path", "launch_count")
+# Names forwarded to the binding: the entry points (ln_*, raw_*), the
+# constants of include/ln.h (LN_*) and the helpers below.  Anything else, the
+# submodules included, is not routed through the binding, so importing
+# ``workloads`` or ``build`` never needs the built library.
+_BINDING_PREFIXES = ("ln_", "LN_", "raw_")
+_BINDING_NAMES = ("LNError", "library_path", "launch_count", "version", "device_status")
 
 
 def __getattr__(name):
-    if name in _BINDING_NAMES:
+    if name.startswith(_BINDING_PREFIXES) or name in _BINDING_NAMES:
         from . import ln
-        return getattr(ln, name)
-    raise AttributeError(name)
+        try:
+            return getattr(ln, name)
+        except AttributeError:
+            pass
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

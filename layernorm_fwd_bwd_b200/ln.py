@@ -138,8 +138,8 @@ def ln_backward(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N: int,
 def ln_forward_residual(resid_out, out, mean, rstd, resid, branch, weight, bias, N: int,
                         C: int, eps: float, dtype: int, stream=None) -> None:
     """resid_out <- resid + branch (rounded to dtype); out, mean, rstd <-
-    LayerNorm(resid_out; weight, bias, eps).  No output may overlap an
-    input."""
+    LayerNorm(resid_out; weight, bias, eps).  No output may overlap another
+    output or an input (LN_ERR_ALIAS)."""
     _check(_lib.ln_forward_residual(_ptr(resid_out), _ptr(out), _ptr(mean), _ptr(rstd),
                                     _ptr(resid), _ptr(branch), _ptr(weight), _ptr(bias),
                                     int(N), int(C), float(eps), int(dtype), _stream(stream)))

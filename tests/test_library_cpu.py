@@ -241,3 +241,19 @@ def test_tolerance_helpers():
     tol.check("x", ref + np.array([2.0 ** -9, 0, 0]), ref, "f16", "act_fwd")
     with pytest.raises(AssertionError):
         tol.check("x", ref + np.array([2.0 ** -8 * 1.01, 0, 0]), ref, "f16", "act_fwd")
+
+
+def test_package_forwards_the_binding(lib):
+    """Every public name of the binding is reachable from the package."""
+    import layernorm_fwd_bwd_b200 as pkg
+    public = [n for n in vars(lib) if not n.startswith("_") and (
+        n.startswith(("ln_", "LN_", "raw_")) or n in pkg._BINDING_NAMES)]
+    for n in ("ln_forward_residual", "ln_backward_ex", "ln_backward_noalloc", "LN_F16",
+              "LN_BWD_RECOMPUTE_STATS", "device_status"):
+        assert n in public
+    for n in public:
+        assert getattr(pkg, n) is getattr(lib, n), n
+    with pytest.raises(AttributeError):
+        pkg.ln_no_such_entry
+    with pytest.raises(AttributeError):
+        pkg.no_such_name
