@@ -36,6 +36,9 @@ LN_BWD_ACCUMULATE_DPARAMS = 2
 LN_BWD_RECOMPUTE_STATS = 4
 LN_NOALLOC_SCRATCH_BYTES = 4 << 20
 LN_NOALLOC_MAX_C = LN_NOALLOC_SCRATCH_BYTES // 8
+LN_MAX_C = 1 << 24
+LN_MAX_N = 1 << 40
+LN_MAX_ELEMS = 1 << 50
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(

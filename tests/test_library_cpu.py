@@ -58,6 +58,7 @@ def test_host_validation_without_gpu(lib):
     # Each of these returns before the library touches the CUDA runtime.
     f = lib.raw_forward
     nz = 16  # any non-NULL address: never dereferenced on these paths
+    n0 = lib.launch_count()   # per process: GPU tests may have run before
     assert f(nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, None) == lib.LN_ERR_SHAPE
     assert f(nz, nz, nz, nz, nz, nz, 4, 0, 1e-5, 0, None) == lib.LN_ERR_SHAPE
     assert f(nz, nz, nz, nz, nz, nz, 4, (1 << 24) + 1, 1e-5, 0, None) == lib.LN_ERR_SHAPE
@@ -74,13 +75,14 @@ def test_host_validation_without_gpu(lib):
     assert b(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 7, None) == lib.LN_ERR_DTYPE
     assert b(nz, None, nz, nz, nz, nz, nz, nz, 4, 8, 0, None) == lib.LN_ERR_NULL
     assert b(nz, nz, None, nz, nz, nz, nz, nz, 0, 8, 0, None) == lib.LN_ERR_NULL
-    assert lib.launch_count() == 0
+    assert lib.launch_count() == n0
 
 
 def test_variant_validation_without_gpu(lib):
     # ln_forward_residual and ln_backward_ex validate like the plain calls,
     # plus their own arguments, before any CUDA call.
     nz = 16
+    n0 = lib.launch_count()
     r = lib.raw_forward_residual
     assert r(nz, nz, nz, nz, nz, nz, nz, nz, -1, 8, 1e-5, 0, None) == lib.LN_ERR_SHAPE
     assert r(nz, nz, nz, nz, nz, nz, nz, nz, 4, 8, 1e-5, 5, None) == lib.LN_ERR_DTYPE
@@ -107,13 +109,14 @@ def test_variant_validation_without_gpu(lib):
     # N == 0 with accumulated parameters has nothing to do (no memset either)
     assert x(None, nz, nz, None, None, None, None, None, 0, 8, 0.0, 0,
              lib.LN_BWD_ACCUMULATE_DPARAMS, None) == lib.LN_OK
-    assert lib.launch_count() == 0
+    assert lib.launch_count() == n0
 
 
 def test_overlapping_outputs_are_refused_without_gpu(lib):
     """Outputs that overlap inputs where the header forbids it return
     LN_ERR_ALIAS before any CUDA call (addresses are never dereferenced; every
     case here is refused on the host, so none can reach a device)."""
+    n0 = lib.launch_count()
     N, C = 4, 8
     act = N * C * 2                      # bytes of one bf16 activation array
     a, b, c, d = 1 << 20, 2 << 20, 3 << 20, 4 << 20   # disjoint fake device addresses
@@ -131,7 +134,7 @@ def test_overlapping_outputs_are_refused_without_gpu(lib):
     x = lib.raw_backward_ex
     assert x(a, c, c + 64, a, b, d, None, None, N, C, 1e-5, 1, lib.LN_BWD_RECOMPUTE_STATS,
              None) == lib.LN_ERR_ALIAS
-    assert lib.launch_count() == 0
+    assert lib.launch_count() == n0
 
 
 def test_every_output_overlap_is_refused_without_gpu(lib):
@@ -139,6 +142,7 @@ def test_every_output_overlap_is_refused_without_gpu(lib):
     call reads: the statistics, the parameter gradients and the small arrays
     included.  Each case starts from a layout of disjoint fake addresses and
     moves one array onto another; all are refused on the host."""
+    n0 = lib.launch_count()
     N, C = 4, 8
     act, par, stat, grad = N * C * 2, C * 2, N * 4, C * 4     # bf16 sizes in bytes
     base = 1 << 20
@@ -204,7 +208,7 @@ def test_every_output_overlap_is_refused_without_gpu(lib):
         lib.ln_backward_noalloc(p["dinp"], p["dweight"], p["dbias"], p["dout"], p["inp"],
                                 p["weight"], p["mean"], p["rstd"], N, C, lib.LN_BF16)
     assert e.value.status == lib.LN_ERR_ALIAS
-    assert lib.launch_count() == 0
+    assert lib.launch_count() == n0
 
 
 def test_binding_raises_lnerror(lib):
@@ -257,3 +261,21 @@ def test_package_forwards_the_binding(lib):
         pkg.ln_no_such_entry
     with pytest.raises(AttributeError):
         pkg.no_such_name
+
+
+def test_binding_constants_match_the_header(lib):
+    """Every LN_* constant of the binding has the value include/ln.h gives it,
+    read by compiling a small C program against the header."""
+    from layernorm_fwd_bwd_b200 import build
+    names = sorted(n for n in vars(lib) if n.startswith("LN_"))
+    assert {"LN_MAX_C", "LN_F16", "LN_ERR_ALIAS", "LN_BWD_RECOMPUTE_STATS"} <= set(names)
+    prints = "".join(f'printf("{n} %lld\\n", (long long)({n}));' for n in names)
+    src = f"#include <stdio.h>\n#include \"ln.h\"\nint main(void) {{ {prints} return 0; }}\n"
+    os.makedirs(build.BUILD_DIR, exist_ok=True)
+    exe = os.path.join(build.BUILD_DIR, "ln_header_constants")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-x", "c", "-", "-o", exe], input=src, text=True, check=True)
+    got = dict(line.split() for line in
+               subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+               if line)
+    assert {n: int(v) for n, v in got.items()} == {n: getattr(lib, n) for n in names}

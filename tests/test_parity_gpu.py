@@ -112,6 +112,78 @@ def test_shape_sweep(lib, dtype, C, N):
     _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_widest_row(lib, dtype):
+    """C = LN_MAX_C (2^24 channels, 32 or 64 MB a row), two rows, every
+    element: rows past every vectorised variant take the scalar kernels with
+    one block per row, and the backward's workspace bound leaves it two
+    blocks."""
+    C = lib.LN_MAX_C
+    batch = wl.custom(dtype, 2, C, seed=24)
+    label = f"{dtype} 2x{C}"
+    dev, _, ref_stats, res = _forward_parity(lib, batch, label, scaled=True)
+    res += _backward_parity(lib, batch, dev, label, ref_stats, scaled=True)
+    print(res)
+
+
+# (dtype, C, rows of one period P, periods k): N * C = k * P * C > 2^31
+BEYOND_INT32 = [("bf16", 768, 4096, 700),    # tile forward, ring backward
+                ("f32", 768, 4096, 700),     # the same kernels, 8.8 GB arrays
+                ("bf16", 770, 4096, 700),    # scalar kernels (C * 2 not a multiple of 16)
+                ("bf16", 4096, 1024, 520),   # two-warp tile forward, register-resident backward
+                ("bf16", 16000, 256, 560)]   # register-resident kernels, 16 warps per row
+
+
+@pytest.mark.parametrize("dtype,C,P,k", BEYOND_INT32)
+def test_beyond_int32_elements(lib, dtype, C, P, k):
+    """More than 2^31 elements per array (element and byte offsets past 32
+    bits).  The rows repeat with period P (the first P rows copied k times on
+    the device), which fixes the result at any size: every output row equals
+    the same row of the first period bit for bit, the first period matches
+    the oracle, and dweight/dbias equal k times the first period's oracle
+    sums.  The backward gets the oracle's statistics rounded to fp32."""
+    N = P * k
+    assert N * C > 2 ** 31
+    batch = wl.custom(dtype, P, C, seed=2 ** 31 + C, dout_sigma=0.02)
+    inp_p, wt, bs, dout_p = gu.batch_to_device(batch)
+    ref_out, ref_mean, ref_rstd = oracle.ln_forward(batch.f64("inp"), batch.f64("weight"),
+                                                    batch.f64("bias"), batch.eps)
+    m32, r32 = ref_mean.astype(np.float32), ref_rstd.astype(np.float32)
+    r_dinp, r_dw, r_db = oracle.ln_backward(batch.f64("dout"), batch.f64("inp"),
+                                            batch.f64("weight"), m32, r32)
+    sc = _scales(batch, m32, r32)
+
+    def periodic(name, t):
+        b = gu.bits(t).reshape(k, -1)
+        for a in range(0, k, 64):
+            assert bool((b[a:a + 64] == b[0]).all()), f"{name}: period {a}.. differs"
+
+    label = f"{dtype} {N}x{C}"
+    inp = inp_p.repeat(k, 1)
+    out, mean, rstd = gu.forward(lib, inp, wt, bs, N, C, batch.eps, dtype)
+    for name, t in (("out", out), ("mean", mean), ("rstd", rstd)):
+        periodic(name, t)
+    res = [tol.check(f"{label} out", gu.to_f64(out[:P]), ref_out, dtype, "act_fwd"),
+           tol.check(f"{label} mean", gu.to_f64(mean[:P]), ref_mean, dtype, "stats",
+                     sc["mean"]),
+           tol.check(f"{label} rstd", gu.to_f64(rstd[:P]), ref_rstd, dtype, "stats")]
+    del out
+    dout = dout_p.repeat(k, 1)
+    dinp, dw, db = gu.backward(lib, dout, inp, wt, torch.from_numpy(m32).cuda().repeat(k),
+                               torch.from_numpy(r32).cuda().repeat(k), N, C, dtype)
+    periodic("dinp", dinp)
+    res += [tol.check(f"{label} dinp", gu.to_f64(dinp[:P]), r_dinp, dtype, "act_bwd",
+                      sc["dinp"]),
+            tol.check(f"{label} dweight", gu.to_f64(dw), k * r_dw, dtype, "param_grad",
+                      k * sc["dweight"]),
+            tol.check(f"{label} dbias", gu.to_f64(db), k * r_db, dtype, "param_grad",
+                      k * sc["dbias"])]
+    assert lib.device_status() == 0
+    print(res)
+    del inp, dout, dinp, mean, rstd
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", [768, 1600, 5])
 def test_misaligned_pointers(lib, dtype, C):
@@ -370,5 +442,13 @@ def test_aliased_outputs_refused(lib):
     assert e.value.status == lib.LN_ERR_ALIAS
     with pytest.raises(lib.LNError) as e:
         lib.ln_forward_residual(x, x.clone(), m, r, x, x.clone(), w, w, N, C, 1e-5, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    # outputs that overlap each other: mean == rstd; dweight == dbias
+    y = torch.empty_like(x)
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_forward(y, m, m, x, w, w, N, C, 1e-5, lib.LN_BF16)
+    assert e.value.status == lib.LN_ERR_ALIAS
+    with pytest.raises(lib.LNError) as e:
+        lib.ln_backward(y, dw, dw, x, x.clone(), w, m, r, N, C, lib.LN_BF16)
     assert e.value.status == lib.LN_ERR_ALIAS
     assert lib.launch_count() == n0
