@@ -1,0 +1,248 @@
+// host_geometry.cu -- host-side check of the library's kernel selection and
+// launch geometry.  It runs on a machine without a GPU: nothing here calls
+// the CUDA runtime, launches a kernel or instantiates one.
+//
+// For every row width the vectorised paths serve (1..2100 16-byte vectors),
+// every element type and every variant, it visits the selection exactly as
+// the launchers do (lnk::visit_fwd_vec, lnk::visit_bwd_ring,
+// lnk::visit_bwd_vec) and checks:
+//   - the chosen variant covers the row, with the fewest vectors per lane
+//     (one-warp rows) or the fewest warps per row (shared rows);
+//   - each family serves exactly its range: one-warp tiles up to 8 vectors
+//     per lane, two-warp tiles up to 16, the backward ring up to its limits,
+//     the register-resident kernels beyond, nothing past 2048 vectors;
+//   - the variant's shared memory fits in one block, for the tile kernels
+//     also with the one-tile and register-resident fallbacks the launcher
+//     may take;
+//   - the ring has 2..8 stages (its 128-byte barrier area holds 16) and
+//     whole row groups of consumer warps.
+// It also compares lnh::tile_rows_per_block with a brute-force search.
+//
+// Output: "sel <fwd|bwd> <dtype> <mode> <first nvec> <last nvec> <variant>"
+// for each run of widths with the same choice, one "FAIL ..." line per
+// failed check, and "checks <n> failures <m>".  Exit status 1 on failure.
+#include <cstdint>
+#include <cstdio>
+#include <string>
+#include <vector>
+
+#include "../layernorm_fwd_bwd_b200/csrc/ln_dispatch.cuh"
+
+namespace {
+
+std::vector<std::string> g_fail;
+long g_checks = 0;
+
+void check(bool ok, const std::string &what) {
+    ++g_checks;
+    if (!ok) g_fail.push_back(what);
+}
+
+template <typename T> const char *tname();
+template <> const char *tname<float>() { return "f32"; }
+template <> const char *tname<lnk::bf16>() { return "bf16"; }
+template <> const char *tname<lnk::f16>() { return "f16"; }
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+std::string num(long v) { return std::to_string(v); }
+
+constexpr size_t kMax = lnk::kMaxSmemPerBlock;
+constexpr int kMaxVec = 16 * 32 * 4;     // widest row of the register-resident kernels
+constexpr int kWidest = 2100;            // widths visited: past kMaxVec
+
+template <typename T, int MODE>
+struct FwdChoice {
+    int nvec;
+    std::string label;
+    static constexpr int E = lnk::Vec<T>::E;
+    static constexpr int kArrays = (MODE & lnk::kFwdResidual) ? 2 : 1;
+
+    std::string ctx() const {
+        return std::string("fwd ") + tname<T>() + " mode " + num(MODE) + " nvec " + num(nvec) +
+               ": ";
+    }
+    // W == 1: the one-warp tile kernel (the launcher takes the
+    // register-resident kernel instead only past 2^34 rows); W > 1: the
+    // register-resident kernel.
+    template <int V, int W, int G>
+    void run() {
+        const int C = nvec * E;
+        if (W == 1) {
+            label = "tile V=" + num(V) + " W=1";
+            check(V == cdiv(nvec, 32), ctx() + "one-warp rows take the fewest vectors per lane");
+            check(V < LN_TILE_FWD_W2_FROM_V, ctx() + "one-warp tiles stay below the two-warp split");
+            check(lnk::fwd_tile_smem<T, lnk::kTileWarps, lnk::kTileFwdTiles, 1, kArrays>(C) <= kMax,
+                  ctx() + "tile shared memory fits");
+            check(lnk::fwd_vec_smem<1, G>(C) <= kMax, ctx() + "register-resident fallback fits");
+        } else {
+            label = "vec V=" + num(V) + " W=" + num(W);
+            check(32 * W * V >= nvec, ctx() + "register-resident rows are covered");
+            check(W == 4 || 32 * (W / 2) * V < nvec,
+                  ctx() + "register-resident rows take the fewest warps");
+            check(!LN_TILE_FWD_TWO_WARPS || nvec > 2 * 32 * 8,
+                  ctx() + "rows of up to 16 vectors per lane take the two-warp tile");
+            check(lnk::fwd_vec_smem<W, G>(C) <= kMax, ctx() + "register-resident smem fits");
+        }
+    }
+    template <int V>
+    void run_tile_two() {
+        const int C = nvec * E;
+        constexpr int NW = 2 * lnk::kTileWarps;
+        label = "tile2 V=" + num(V) + " W=2";
+        if (lnk::fwd_tile_smem<T, NW, lnk::kTileFwdTiles, 2, kArrays>(C) > kMax)
+            label += " tiles=1";
+        check(64 * V >= nvec && 64 * (V - 1) < nvec,
+              ctx() + "two-warp rows take the fewest vectors per lane");
+        check(nvec > 32 * 8, ctx() + "two-warp rows are wider than one warp serves");
+        check(lnk::fwd_tile_smem<T, NW, 1, 2, kArrays>(C) <= kMax,
+              ctx() + "a one-tile two-warp block fits");
+        check(nvec <= 4 * 32 * 4 && lnk::fwd_vec_smem<4, 2>(C) <= kMax,
+              ctx() + "the four-warp register-resident fallback covers the row");
+    }
+};
+
+template <typename T, int MODE>
+struct BwdChoice {
+    int nvec;
+    std::string label;
+    static constexpr int E = lnk::Vec<T>::E;
+    static constexpr int NS = lnk::BwdRingArrays<MODE>::value;
+    static constexpr int ONE = lnk::RingVmax<T, MODE>::one;
+    static constexpr int VS = lnk::RingVmax<T, MODE>::shared;
+
+    std::string ctx() const {
+        return std::string("bwd ") + tname<T>() + " mode " + num(MODE) + " nvec " + num(nvec) +
+               ": ";
+    }
+    template <int V, int W>
+    void ring() {
+        const int C = nvec * E;
+        constexpr int NC = lnk::BwdRingConsumers<W>::value;
+        constexpr int S = lnk::BwdStages<V, NC, NS>::value;
+        label = "ring V=" + num(V) + " W=" + num(W) + " S=" + num(S);
+        check(32 * W * V >= nvec, ctx() + "ring rows are covered");
+        if (W == 1)
+            check(V == cdiv(nvec, 32) && V <= ONE,
+                  ctx() + "one-warp ring rows take the fewest vectors per lane");
+        else
+            check(V == VS && W == cdiv(nvec, 32 * VS) && nvec > 32 * ONE,
+                  ctx() + "shared ring rows: the fixed vectors per lane, the fewest warps, "
+                          "only past one warp's reach");
+        check(S >= 2 && S <= 8, ctx() + "ring depth 2..8");
+        check(NC % W == 0 && NC >= W, ctx() + "whole row groups of consumer warps");
+        check(lnk::bwd_tma_smem<T, NC, S, W, NS>(C) <= kMax, ctx() + "ring shared memory fits");
+    }
+    template <int V, int W, int G>
+    void run() {
+        const int C = nvec * E;
+        label = "vec V=" + num(V) + " W=" + num(W);
+        check(nvec > 4 * 32 * VS && nvec > 32 * ONE,
+              ctx() + "the register-resident backward serves only rows past the ring");
+        check(32 * W * V >= nvec, ctx() + "register-resident rows are covered");
+        check(W == 4 || 32 * (W / 2) * V < nvec,
+              ctx() + "register-resident rows take the fewest warps");
+        check(lnk::bwd_vec_smem<W, G>(C) <= kMax, ctx() + "register-resident smem fits");
+    }
+};
+
+// Prints each run of widths that share a choice.
+struct Runs {
+    std::string head, label;
+    int first = 0, last = 0;
+    void add(int nvec, const std::string &l) {
+        if (!label.empty() && l == label && nvec == last + 1) {
+            last = nvec;
+            return;
+        }
+        flush();
+        label = l;
+        first = last = nvec;
+    }
+    void flush() {
+        if (!label.empty())
+            std::printf("sel %s %d %d %s\n", head.c_str(), first, last, label.c_str());
+        label.clear();
+    }
+};
+
+template <typename T, int MODE>
+void forward_all() {
+    Runs runs{std::string("fwd ") + tname<T>() + " " + num(MODE)};
+    for (int nvec = 1; nvec <= kWidest; ++nvec) {
+        FwdChoice<T, MODE> c{nvec, ""};
+        const bool found = lnk::visit_fwd_vec<T>(nvec, c);
+        check(found == (nvec <= kMaxVec),
+              c.ctx() + "a vectorised forward exists exactly up to 2048 vectors");
+        runs.add(nvec, found ? c.label : std::string("scalar"));
+    }
+    runs.flush();
+}
+
+template <typename T, int MODE>
+void backward_all() {
+    Runs runs{std::string("bwd ") + tname<T>() + " " + num(MODE)};
+    for (int nvec = 1; nvec <= kWidest; ++nvec) {
+        BwdChoice<T, MODE> c{nvec, ""};
+        bool found = lnk::visit_bwd_ring<T, MODE>(nvec, c);
+        if (!found) found = lnk::visit_bwd_vec<T>(nvec, c);
+        check(found == (nvec <= kMaxVec),
+              c.ctx() + "a vectorised backward exists exactly up to 2048 vectors");
+        runs.add(nvec, found ? c.label : std::string("scalar"));
+    }
+    runs.flush();
+}
+
+void rows_per_block_all() {
+    const int64_t Ns[] = {1, 7, 8, 9, 100, 4097, 16384, 32768, 65536, 1000003,
+                          int64_t(1) << 34};
+    const int64_t residents[] = {1, 148, 296, 444, 592, 1184};
+    for (int64_t N : Ns)
+        for (int max_rows : {8, 16})
+            for (int64_t res : residents) {
+                const int got = lnh::tile_rows_per_block(N, max_rows, res);
+                // fewest rows in total (whole waves of `res` blocks times rows
+                // per block); among equals, more rows per block
+                int want = 0;
+                int64_t want_cost = 0;
+                for (int rows = (max_rows + 1) / 2; rows <= max_rows; ++rows) {
+                    const int64_t blocks = (N + rows - 1) / rows;
+                    const int64_t cost = (blocks + res - 1) / res * rows;
+                    if (want == 0 || cost <= want_cost) {
+                        want = rows;
+                        want_cost = cost;
+                    }
+                }
+                check(got == want, "tile_rows_per_block(" + num(N) + ", " + num(max_rows) + ", " +
+                                       num(res) + ") = " + num(got) + ", brute force " +
+                                       num(want));
+            }
+    check(lnh::tile_rows_per_block(16384, 16, 444) == 13,
+          "GPT-2 1.5B forward: 13 rows per block on 444 resident blocks");
+}
+
+}  // namespace
+
+int main() {
+    forward_all<float, 0>();
+    forward_all<float, lnk::kFwdResidual>();
+    forward_all<lnk::bf16, 0>();
+    forward_all<lnk::bf16, lnk::kFwdResidual>();
+    forward_all<lnk::f16, 0>();
+    forward_all<lnk::f16, lnk::kFwdResidual>();
+    backward_all<float, 0>();
+    backward_all<float, lnk::kBwdAccumulate>();
+    backward_all<float, lnk::kBwdRecompute>();
+    backward_all<float, lnk::kBwdAccumulate | lnk::kBwdRecompute>();
+    backward_all<lnk::bf16, 0>();
+    backward_all<lnk::bf16, lnk::kBwdAccumulate>();
+    backward_all<lnk::bf16, lnk::kBwdRecompute>();
+    backward_all<lnk::bf16, lnk::kBwdAccumulate | lnk::kBwdRecompute>();
+    backward_all<lnk::f16, 0>();
+    backward_all<lnk::f16, lnk::kBwdAccumulate>();
+    backward_all<lnk::f16, lnk::kBwdRecompute>();
+    backward_all<lnk::f16, lnk::kBwdAccumulate | lnk::kBwdRecompute>();
+    rows_per_block_all();
+    for (const std::string &f : g_fail) std::printf("FAIL %s\n", f.c_str());
+    std::printf("checks %ld failures %zu\n", g_checks, g_fail.size());
+    return g_fail.empty() ? 0 : 1;
+}
