@@ -8,7 +8,10 @@ libcudart the host process (for example PyTorch) has loaded.
 
 The kernels are compiled in parallel, one object per (direction, element type,
 variant) from ``csrc/ln_inst.cu``, plus the API and no-alloc units; objects go
-to ``_build/`` beside this file and are linked into the one library.
+to ``_build/`` beside this file and are linked into the one library.  ptxas
+reports each kernel's registers, stack and spills (``-Xptxas=-v``, which only
+prints); the report of each object is kept beside it as ``<object>.ptxas.txt``
+(``--verbose`` also prints it).
 """
 from __future__ import annotations
 
@@ -53,10 +56,18 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPENDS)
 
 
-def _jobs(verbose: bool) -> list[tuple[str, list[str]]]:
-    base = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE]
-    if verbose:
-        base.insert(1, "-Xptxas=-v")
+def ptxas_report(obj: str) -> str:
+    """Path of the ptxas resource report kept for one object."""
+    return obj + ".ptxas.txt"
+
+
+def objects() -> list[str]:
+    """Every object the library links."""
+    return [obj for obj, _ in _jobs()]
+
+
+def _jobs() -> list[tuple[str, list[str]]]:
+    base = [nvcc(), *NVCC_FLAGS, "-Xptxas=-v", "-I", INCLUDE]
     jobs = []
     for unit in UNITS:
         obj = os.path.join(BUILD_DIR, unit.replace(".cu", ".o"))
@@ -72,7 +83,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
     if not force and not stale():
         return LIBRARY
     os.makedirs(BUILD_DIR, exist_ok=True)
-    jobs = _jobs(verbose)
+    jobs = _jobs()
 
     def compile_one(job):
         return subprocess.run(job[1], capture_output=True, text=True)
@@ -85,6 +96,9 @@ def build(verbose: bool = False, force: bool = False) -> str:
         if verbose or res.returncode != 0:
             sys.stderr.write(f"== {os.path.basename(obj)}\n{res.stdout}{res.stderr}")
         failed |= res.returncode != 0
+        if res.returncode == 0:
+            with open(ptxas_report(obj), "w") as f:
+                f.write(res.stdout + res.stderr)
     if failed:
         raise RuntimeError("nvcc failed (see the messages above)")
     link = [nvcc(), *LINK_FLAGS, "-o", LIBRARY + ".tmp", *[obj for obj, _ in jobs]]
