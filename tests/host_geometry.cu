@@ -15,7 +15,10 @@
 //     also with the one-tile and register-resident fallbacks the launcher
 //     may take;
 //   - the ring has 2..8 stages (its 128-byte barrier area holds 16) and
-//     whole row groups of consumer warps.
+//     whole row groups of consumer warps;
+//   - every bulk copy is a whole number of 16-byte units, and the bytes one
+//     mbarrier phase expects (all the copies that complete on it) stay below
+//     the 2^20 limit of an mbarrier's transaction count.
 // It also compares lnh::tile_rows_per_block with a brute-force search.
 //
 // Output: "sel <fwd|bwd> <dtype> <mode> <first nvec> <last nvec> <variant>"
@@ -47,6 +50,15 @@ int cdiv(int a, int b) { return (a + b - 1) / b; }
 std::string num(long v) { return std::to_string(v); }
 
 constexpr size_t kMax = lnk::kMaxSmemPerBlock;
+constexpr size_t kMaxTx = (size_t(1) << 20) - 1;   // mbarrier transaction count limit
+
+// The bulk copies of a tile or stage: `arrays` copies of `rows` rows of
+// `row_bytes` each, all completing on one mbarrier phase.
+void check_copies(const std::string &ctx, size_t row_bytes, int rows, int arrays) {
+    check(row_bytes % 16 == 0, ctx + "bulk copies are whole 16-byte units");
+    check(size_t(arrays) * rows * row_bytes <= kMaxTx,
+          ctx + "one phase expects fewer than 2^20 bytes");
+}
 constexpr int kMaxVec = 16 * 32 * 4;     // widest row of the register-resident kernels
 constexpr int kWidest = 2100;            // widths visited: past kMaxVec
 
@@ -73,6 +85,8 @@ struct FwdChoice {
             check(V < LN_TILE_FWD_W2_FROM_V, ctx() + "one-warp tiles stay below the two-warp split");
             check(lnk::fwd_tile_smem<T, lnk::kTileWarps, lnk::kTileFwdTiles, 1, kArrays>(C) <= kMax,
                   ctx() + "tile shared memory fits");
+            check_copies(ctx(), size_t(C) * sizeof(T), lnk::kTileWarps, kArrays);
+            check_copies(ctx() + "weight and bias: ", size_t(C) * sizeof(T), 1, 2);
             check(lnk::fwd_vec_smem<1, G>(C) <= kMax, ctx() + "register-resident fallback fits");
         } else {
             label = "vec V=" + num(V) + " W=" + num(W);
@@ -96,6 +110,8 @@ struct FwdChoice {
         check(nvec > 32 * 8, ctx() + "two-warp rows are wider than one warp serves");
         check(lnk::fwd_tile_smem<T, NW, 1, 2, kArrays>(C) <= kMax,
               ctx() + "a one-tile two-warp block fits");
+        check_copies(ctx(), size_t(C) * sizeof(T), NW / 2, kArrays);
+        check_copies(ctx() + "weight and bias: ", size_t(C) * sizeof(T), 1, 2);
         check(nvec <= 4 * 32 * 4 && lnk::fwd_vec_smem<4, 2>(C) <= kMax,
               ctx() + "the four-warp register-resident fallback covers the row");
     }
@@ -131,6 +147,7 @@ struct BwdChoice {
         check(S >= 2 && S <= 8, ctx() + "ring depth 2..8");
         check(NC % W == 0 && NC >= W, ctx() + "whole row groups of consumer warps");
         check(lnk::bwd_tma_smem<T, NC, S, W, NS>(C) <= kMax, ctx() + "ring shared memory fits");
+        check_copies(ctx(), size_t(C) * sizeof(T), NC / W, NS);
     }
     template <int V, int W, int G>
     void run() {
