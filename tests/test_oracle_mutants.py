@@ -56,14 +56,19 @@ MUTANTS = [
 ]
 
 
+# the mutants are built inside the repository, in a folder git ignores
+MUTANT_DIR = os.path.join(os.path.dirname(oracle.SOURCE), "_build", "mutants")
+
+
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_mutant(tmp_path, name, old, new):
+def test_pins_catch_mutant(name, old, new):
     src = open(oracle.SOURCE).read()
     assert old in src, f"mutation site for {name} no longer in the oracle source"
-    mutant_src = os.path.join(tmp_path, f"{name}.c")
+    os.makedirs(MUTANT_DIR, exist_ok=True)
+    mutant_src = os.path.join(MUTANT_DIR, f"{name}.c")
     with open(mutant_src, "w") as f:
         f.write(src.replace(old, new))
-    lib = oracle.compile_oracle(mutant_src, os.path.join(tmp_path, f"{name}.so"))
+    lib = oracle.compile_oracle(mutant_src, os.path.join(MUTANT_DIR, f"{name}.so"))
     mutant = oracle.Oracle(library=lib, source=mutant_src)
     caught = []
     for pin in oracle_pins.ALL_PINS:
