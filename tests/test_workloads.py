@@ -1,5 +1,6 @@
 """The seeded input generator (CPU only)."""
 import numpy as np
+import pytest
 
 from layernorm_fwd_bwd_b200 import workloads as wl
 
@@ -58,6 +59,36 @@ def test_compulsory_bytes():
     assert w.bwd_bytes() == 302_521_856
     assert wl.WORKLOADS["stress_fp32_65536x768"].fwd_bytes() + \
         wl.WORKLOADS["stress_fp32_65536x768"].bwd_bytes() == 1_007_696_896
+
+
+@pytest.mark.parametrize("name,fwd,bwd", [
+    ("fp32_256x768", 1_581_056, 2_370_560),
+    ("gpt2_124m_bf16", 201_853_952, 302_521_856),
+    ("gpt2_350m_bf16", 134_483_968, 201_598_976),
+    ("gpt2_1558m_bf16", 104_995_072, 157_433_472),
+    ("stress_fp32_65536x768", 403_183_616, 604_513_280),
+])
+def test_compulsory_bytes_every_workload(name, fwd, bwd):
+    """The per-call byte counts every GB/s figure divides by, against the
+    table computed independently when the workloads were specified."""
+    w = wl.WORKLOADS[name]
+    assert (w.fwd_bytes(), w.bwd_bytes()) == (fwd, bwd)
+
+
+def test_variant_bytes_follow_from_the_plain_calls():
+    """Each variant's compulsory bytes differ from the plain call's by exactly
+    the arrays it adds or drops: the residual forward reads branch and writes
+    resid_out (2NCs more); accumulating reads the previous dinp (NCs) and
+    reads dweight/dbias (8C); recomputing reads no saved statistics (8N
+    fewer)."""
+    import bench
+    for w in wl.WORKLOADS.values():
+        N, C, s = w.N, w.C, w.elem_bytes
+        v = bench.variant_bytes(w)
+        assert v["fwd_residual"] == w.fwd_bytes() + 2 * N * C * s
+        assert v["bwd_accumulate"] == w.bwd_bytes() + N * C * s + 8 * C
+        assert v["bwd_recompute"] == w.bwd_bytes() - 8 * N
+        assert v["bwd_accumulate_recompute"] == w.bwd_bytes() + N * C * s + 8 * C - 8 * N
 
 
 def test_f16_storage_roundtrip():
