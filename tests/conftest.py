@@ -26,13 +26,14 @@ def orc():
 # root cause: the oracle against its pins before anything is compared with
 # it, the input generator, the library's loading and host validation, its
 # resource report, the bounds on every device wait, its kernel selection,
-# the benchmark's rank logic, then GPU parity of the plain calls, of the
-# variants, and last the allocation-free backward.  Files not listed run
-# after the variants; tests keep their order within a file.
+# the benchmark's rank logic and its profile summaries, then GPU parity of
+# the plain calls, of the variants, and last the allocation-free backward.
+# Files not listed run after the variants; tests keep their order within a
+# file.
 _ORDER = ["test_oracle_pins.py", "test_oracle_mutants.py", "test_workloads.py",
           "test_library_cpu.py", "test_build_cpu.py", "test_device_safety_cpu.py",
-          "test_host_geometry.py", "test_bench_multirank.py", "test_parity_gpu.py",
-          "test_variants_gpu.py"]
+          "test_host_geometry.py", "test_bench_multirank.py", "test_profiles_cpu.py",
+          "test_parity_gpu.py", "test_variants_gpu.py"]
 _LAST = "test_zz_no_alloc.py"
 
 
