@@ -2,6 +2,14 @@
 // row tiles into shared memory with TMA bulk copies, uses every stage exactly
 // once, and exits.
 //
+// Operation: the LayerNorm forward of "llm.c's Origin and the Future of LLM
+// Compilers" (CUDA MODE talk page), chapter "Deconstructing PyTorch
+// Abstractions and Setting Reference Baselines", over the flat row-major
+// arrays of "llm.c: Large Language Model Training in Pure C/CUDA Without
+// Dependencies", feature "Tensor Memory Layout"; the residual variant fuses
+// the add before it, as that page's feature list credits custom fused
+// kernels.  Arithmetic as in ln_kernels.cuh.
+//
 // Why one-shot.  Measured on B200 with copy kernels of the LayerNorm access
 // pattern (no arithmetic): short-lived blocks that each move 16 rows reach
 // 5.6 TB/s (forward-shaped, 100 MB in + 100 MB out) and 6.1 TB/s

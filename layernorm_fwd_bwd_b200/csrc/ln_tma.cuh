@@ -2,6 +2,13 @@
 // also used by the one-shot forward in ln_tile.cuh) and the LayerNorm
 // backward fed by a TMA bulk-copy ring.
 //
+// Operation: the hand-derived LayerNorm gradient of "llm.c: Large Language
+// Model Training in Pure C/CUDA Without Dependencies", feature "Exact
+// Analytical Backward Pass" (dinp, and dweight/dbias summed over all rows);
+// the accumulating variant adds into the previous gradients, as that page's
+// multi-GPU question says gradients are accumulated locally.  Arithmetic as
+// in ln_kernels.cuh.
+//
 // Why a ring: the register-resident kernels keep at most one row per warp in flight
 // (1.5 KB for a bf16 row of 768), and a warp spends most of each row on
 // arithmetic, so a bf16 launch cannot keep enough bytes in flight to reach
