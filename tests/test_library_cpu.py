@@ -279,3 +279,58 @@ def test_binding_constants_match_the_header(lib):
                subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
                if line)
     assert {n: int(v) for n, v in got.items()} == {n: getattr(lib, n) for n in names}
+
+
+# C parameter types of include/ln.h and the ctypes type the binding must
+# declare for each
+_CTYPES = {"void *": "c_void_p", "const void *": "c_void_p", "float *": "c_void_p",
+           "const float *": "c_void_p", "int64_t": "c_long", "int": "c_int",
+           "float": "c_float", "unsigned int": "c_uint", "ln_stream_t": "c_void_p",
+           "unsigned int *": "LP_c_uint", "void": None}
+
+
+def _prototypes():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for ret, name, params in re.findall(
+            r"^\s*(int|const char \*|uint64_t)\s*(ln_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M):
+        types = []
+        for p in params.split(","):
+            p = " ".join(p.split())
+            if p in ("void", ""):
+                continue
+            t = re.sub(r"\s*\b\w+$", "", p)          # drop the parameter name
+            types.append(re.sub(r"\s*\*", " *", t).strip())
+        out[name] = (ret, types)
+    return out
+
+
+_RESTYPES = {"int": "c_int", "const char *": "c_char_p", "uint64_t": "c_ulong"}
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every function of include/ln.h is declared to ctypes with the same
+    number of parameters and matching types, so no call passes an argument
+    the library reads as something else."""
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, types) in protos.items():
+        fn = getattr(lib._lib, name)
+        got = [t.__name__ for t in (fn.argtypes or [])]
+        want = [_CTYPES[t] for t in types]
+        # ctypes spells the 64-bit integers c_long / c_ulong on LP64 hosts
+        got = ["c_long" if g in ("c_int64", "c_longlong") else g for g in got]
+        assert got == want, f"{name}: header {types}, binding {got}"
+        res = {"c_uint64": "c_ulong", "c_ulonglong": "c_ulong"}.get(fn.restype.__name__,
+                                                                     fn.restype.__name__)
+        assert res == _RESTYPES[ret], f"{name}: returns {ret}, binding {fn.restype.__name__}"
+
+
+def test_header_compiles_as_cpp():
+    """C++ callers include the same header (extern "C", no warnings)."""
+    src = ('#include "ln.h"\n'
+           'int (*const version)(void) = ln_version;\n'
+           'int main() { return version != ln_version; }\n')
+    subprocess.run(["g++", "-std=c++11", "-Wall", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), "-x", "c++", "-", "-fsyntax-only"],
+                   input=src, text=True, check=True)
