@@ -74,6 +74,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-variants", action="store_true",
                    help="skip timing ln_forward_residual, ln_backward_ex and fp16")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip timing forward and backward on every workload")
     p.add_argument("--sets", type=int, default=SETS,
                    help="rotating buffer sets (>= 2 so a step's backward never "
                         "reads what its forward just read)")
@@ -158,6 +160,21 @@ class ClockSampler:
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+
+    def wait_first_sample(self, timeout: float = 5.0) -> bool:
+        """Block until nvidia-smi has written its first line (it needs about
+        a second to start), so that samples cover the region that follows."""
+        if self.proc is None:
+            return False
+        t_end = time.time() + timeout
+        while time.time() < t_end:
+            self.file.flush()
+            if os.path.getsize(self.file.name) > 0:
+                return True
+            if self.proc.poll() is not None:
+                return False
+            time.sleep(0.05)
+        return False
 
     def stop(self):
         if self.proc is not None:
@@ -292,6 +309,8 @@ def run_ours(args, world: int, rank: int, local: int):
 
     K, W = args.steps, args.warmup
     sampler = ClockSampler(local) if rank == 0 else None
+    if sampler is not None:
+        sampler.wait_first_sample()
     for i in range(W):
         step(i)
     # per-call events on every EVERY-th timed step only: an event record
@@ -315,8 +334,6 @@ def run_ours(args, world: int, rank: int, local: int):
     if world > 1:
         dist.barrier()
     launches = ln.launch_count() - launches0
-    if sampler is not None:
-        sampler.stop()
     total_ms = start.elapsed_time(end)
     fwd_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in events.values())
     bwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in events.values())
@@ -331,6 +348,12 @@ def run_ours(args, world: int, rank: int, local: int):
                                            h_w, h_b, N, C, tdt, dcode, eps, world)
     variants = None if args.no_variants else run_variants(
         torch, ln, stream, sets, weight, bias, dweight, dbias, w, eps, dcode)
+    t_loops = time.time()
+    if sampler is not None:
+        sampler.stop()
+    del sets, fargs, bargs
+    workloads = None if (args.no_workloads or rank != 0) else run_workloads(
+        torch, ln, stream, dev, args.sets)
 
     if world > 1:
         dist.barrier()
@@ -344,7 +367,11 @@ def run_ours(args, world: int, rank: int, local: int):
     peak, peak_kind = hbm_peak()
     bwd_gbs = bb / (bwd_loop_us / 1e6) / 1e9
     fwd_gbs = fb / (fwd_loop_us / 1e6) / 1e9
-    clocks = sampler.summary(t0, t1) if sampler else None
+    clocks = None
+    if sampler:
+        clocks = sampler.summary(t0, t_loops)
+        clocks["window"] = ("from the first timed step to the end of the variant loops: "
+                            "timed steps, fwd/bwd call loops, e2e, variants")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": K, "warmup": W,
@@ -371,11 +398,16 @@ def run_ours(args, world: int, rank: int, local: int):
         "roofline": {"bound": "hbm", "kernel": "ln_backward (row pass + column finalise)",
                      "achieved": round(bwd_gbs, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(bwd_gbs / peak, 4),
-                     "traffic": profiled_traffic()},
+                     "traffic": profiled_traffic(),
+                     "traffic_note": "DRAM bytes (read + write) during one serialised "
+                                     "launch of each of the two kernels under ncu; below the "
+                                     "algorithmic bytes because part of dinp is still dirty "
+                                     "in L2 when a launch ends"},
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
         "variants": variants,
+        "workloads": workloads,
     }
     line["cpu_baseline"] = (None if (world > 1 or args.no_cpu_baseline)
                             else cpu_baseline(w, args.cpu_seconds))
@@ -485,6 +517,85 @@ def run_variants(torch, ln, stream, sets, weight, bias, dweight, dbias, w, eps, 
         gbs = nbytes[name] / (us * 1e-6) / 1e9
         out[name] = {"us": round(us, 3), "GB_s": round(gbs, 1), "bytes": nbytes[name],
                      "frac": round(gbs / peak, 4), "calls": calls}
+    return out
+
+
+def run_workloads(torch, ln, stream, dev, nsets: int, calls: int = LOOP_CALLS) -> dict:
+    """ln_forward and ln_backward on every workload at its full size, each
+    timed like the headline's fwd and bwd: `calls` back-to-back calls over
+    rotating buffer sets (a backward reads a set whose forward ran
+    ``nsets // 2`` calls earlier), CUDA events around the loop on the
+    launching stream.  GB/s counts compulsory bytes; ``frac`` is against the
+    measured HBM copy bandwidth (or the fallback, as ``peak_kind`` says)."""
+    import numpy as np
+
+    from layernorm_fwd_bwd_b200 import workloads as wl
+    peak, _ = hbm_peak()
+    nsets = max(2, nsets)
+    out = {}
+    for name, w in wl.WORKLOADS.items():
+        batch = wl.generate(w)
+        N, C = w.N, w.C
+        tdt = torch.float32 if w.dtype == wl.F32 else torch.bfloat16
+        code = ln.LN_F32 if w.dtype == wl.F32 else ln.LN_BF16
+
+        def dev_t(a):
+            if w.dtype == wl.F32:
+                t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
+            else:
+                t = torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).view(
+                    torch.bfloat16)
+            return t.to(dev, non_blocking=False)
+
+        with torch.cuda.stream(stream):
+            inp, dout = dev_t(batch.inp), dev_t(batch.dout)
+            weight, bias = dev_t(batch.weight), dev_t(batch.bias)
+            dweight, dbias = torch.empty(C, device=dev), torch.empty(C, device=dev)
+            sets = [dict(inp=inp.clone(), dout=dout.clone(),
+                         out=torch.empty(N, C, dtype=tdt, device=dev),
+                         dinp=torch.empty(N, C, dtype=tdt, device=dev),
+                         mean=torch.empty(N, device=dev), rstd=torch.empty(N, device=dev))
+                    for _ in range(nsets)]
+        del inp, dout, batch
+        stream.synchronize()
+        sp = stream.cuda_stream
+        p = lambda t: t.data_ptr()
+
+        def fwd(i):
+            a = sets[i % nsets]
+            rc = ln.raw_forward(p(a["out"]), p(a["mean"]), p(a["rstd"]), p(a["inp"]),
+                                p(weight), p(bias), N, C, 1e-5, code, sp)
+            if rc:
+                raise ln.LNError(rc)
+
+        def bwd(i):
+            b = sets[(i + nsets // 2) % nsets]
+            rc = ln.raw_backward(p(b["dinp"]), p(dweight), p(dbias), p(b["dout"]),
+                                 p(b["inp"]), p(weight), p(b["mean"]), p(b["rstd"]), N, C,
+                                 code, sp)
+            if rc:
+                raise ln.LNError(rc)
+
+        for k in range(nsets):
+            fwd(k)
+        f_us = call_loop_us(torch, stream, fwd, calls)
+        b_us = call_loop_us(torch, stream, bwd, calls)
+        fb, bb = w.fwd_bytes(), w.bwd_bytes()
+        step_gbs = (fb + bb) / ((f_us + b_us) * 1e-6) / 1e9
+        out[name] = {
+            "N": N, "C": C, "dtype": w.dtype,
+            "fwd_us": round(f_us, 3), "bwd_us": round(b_us, 3),
+            "fwd_GB_s": round(fb / (f_us * 1e-6) / 1e9, 1),
+            "bwd_GB_s": round(bb / (b_us * 1e-6) / 1e9, 1),
+            "GB_s": round(step_gbs, 1), "rows_per_s": round(N / ((f_us + b_us) * 1e-6), 1),
+            "frac": round(step_gbs / peak, 4),
+            "bwd_frac": round(bb / (b_us * 1e-6) / 1e9 / peak, 4),
+            "bytes": fb + bb,
+            "l2": ("inputs smaller than L2: launch-bound correctness case"
+                   if nsets * 2 * N * C * w.elem_bytes < 126e6 else
+                   f"{nsets} rotating sets, inputs never re-read from L2")}
+        del sets
+        torch.cuda.empty_cache()
     return out
 
 
@@ -607,6 +718,7 @@ def cpu_baseline(w, seconds: float) -> dict:
     rows = min(w.N, 16384)
     gbs, per, reps = _oracle_rate(w, rows, seconds)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "host_cores": os.cpu_count(),
             "sample": f"first {rows} of {w.N} rows of {w.name}, forward+backward in "
                       f"double, median of {reps} passes ({per:.3f} s each), "
                       "single thread"}
@@ -655,7 +767,7 @@ def run_reference(args, world: int, rank: int):
         "config": {"workload": w.name, "description": w.description, "N": w.N, "C": w.C,
                    "activations": w.dtype, "rows_per_step_sample": rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
-                         "kind": "oracle", "sample": sample},
+                         "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -239,7 +239,31 @@ uint64_t ln_launch_count(void);
  * the current device.  Returns LN_OK, LN_ERR_NULL or LN_ERR_CUDA. */
 int ln_device_status(unsigned int *bits, int clear);
 
-/* Library ABI version: 2 (1 plus ln_forward_residual, ln_backward_ex and
+/*
+ * Caps the workspace that one ln_backward or ln_backward_ex call on the
+ * current device may draw from the pool, in bytes (0, the default: no cap).
+ * A call that needs more (G * 2 * C * 4 bytes, G the backward's grid, about
+ * the SM count) returns LN_ERR_WORKSPACE before launching anything, exactly
+ * as when the pool cannot supply it; the setting stays until changed, and
+ * later calls that fit run normally.  For callers that budget device memory
+ * per library, and for exercising the workspace-failure path without
+ * exhausting a shared GPU.  ln_backward_noalloc is not affected.  Returns
+ * LN_OK, LN_ERR_SHAPE for bytes < 0, or LN_ERR_CUDA.
+ */
+int ln_set_workspace_limit(int64_t bytes);
+
+/*
+ * The CUDA error behind the most recent LN_ERR_CUDA returned on the calling
+ * host thread: its name, number and description, and the runtime call that
+ * raised it (for example "cudaErrorInvalidValue (1: invalid argument) in
+ * cudaLaunchKernelEx").  Never NULL; the text is owned by the library and
+ * stays valid until the thread's next failing call.  Calls that succeed do
+ * not reset it.
+ */
+const char *ln_last_cuda_error(void);
+
+/* Library ABI version: 3 (2 plus ln_set_workspace_limit and
+ * ln_last_cuda_error; 2 was 1 plus ln_forward_residual, ln_backward_ex and
  * LN_F16). */
 int ln_version(void);
 

@@ -15,7 +15,8 @@ without the library raises immediately (there is no CPU fallback).
 # submodules included, is not routed through the binding, so importing
 # ``workloads`` or ``build`` never needs the built library.
 _BINDING_PREFIXES = ("ln_", "LN_", "raw_")
-_BINDING_NAMES = ("LNError", "library_path", "launch_count", "version", "device_status")
+_BINDING_NAMES = ("LNError", "library_path", "launch_count", "version", "device_status",
+                  "last_cuda_error", "set_workspace_limit")
 
 
 def __getattr__(name):

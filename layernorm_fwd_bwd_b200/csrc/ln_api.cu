@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 #include <unordered_map>
 
@@ -27,9 +28,15 @@ static __device__ unsigned int ln_status_word;
 struct DeviceState {
     std::once_flag once;
     int sms = 0;
-    cudaMemPool_t pool = nullptr;
     unsigned int *status = nullptr;   // device address of ln_status_word
     cudaError_t init_error = cudaSuccess;
+    // The workspace pool of ln_backward / ln_backward_ex, created on the
+    // first pooled call only, so that a process that only ever calls
+    // ln_backward_noalloc never creates one.
+    std::once_flag pool_once;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t pool_error = cudaSuccess;
+    std::atomic<uint64_t> workspace_limit{0};   // bytes per call; 0: no cap
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -38,17 +45,6 @@ cudaError_t device_state(int dev, DeviceState **out) {
     DeviceState &d = g_dev[dev];
     std::call_once(d.once, [&]() {
         cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess) {
-            cudaMemPoolProps props = {};
-            props.allocType = cudaMemAllocationTypePinned;
-            props.location.type = cudaMemLocationTypeDevice;
-            props.location.id = dev;
-            e = cudaMemPoolCreate(&d.pool, &props);
-        }
-        if (e == cudaSuccess) {
-            uint64_t keep = UINT64_MAX;
-            e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        }
         if (e == cudaSuccess)
             e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), ln_status_word);
         d.init_error = e;
@@ -56,6 +52,15 @@ cudaError_t device_state(int dev, DeviceState **out) {
     *out = &d;
     return d.init_error;
 }
+
+// The last CUDA error behind an LN_ERR_CUDA on this host thread, and the
+// call that raised it.
+struct LastCudaError {
+    cudaError_t code = cudaSuccess;
+    const char *call = "";
+};
+thread_local LastCudaError t_last_error;
+thread_local char t_last_error_text[256];
 
 // Occupancy (resident blocks per SM) per kernel, device, block size and
 // dynamic shared memory size.
@@ -78,10 +83,28 @@ std::mutex g_occ_mu;
 std::unordered_map<OccKey, int, OccHash> g_occ;
 
 int current_device(int *dev, DeviceState **ds) {
-    if (cudaGetDevice(dev) != cudaSuccess) return LN_ERR_CUDA;
-    if (device_state(*dev, ds) != cudaSuccess) return LN_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return lnh::note_cuda_error(e, "cudaGetDevice");
+    e = device_state(*dev, ds);
+    if (e != cudaSuccess)
+        return lnh::note_cuda_error(e, "device set-up (SM count, status word address)");
     return LN_OK;
 }
+
+// Smallest dynamic shared-memory limit known to be in force per kernel and
+// device (raised by raise_smem_limit, never lowered).
+struct FnDev {
+    const void *fn;
+    int dev;
+    bool operator==(const FnDev &o) const { return fn == o.fn && dev == o.dev; }
+};
+struct FnDevHash {
+    size_t operator()(const FnDev &k) const {
+        return std::hash<const void *>()(k.fn) ^ (size_t(k.dev) << 1);
+    }
+};
+std::mutex g_smem_mu;
+std::unordered_map<FnDev, size_t, FnDevHash> g_smem_limit;
 
 int check_shape(int64_t N, int64_t C) {
     if (N < 0 || N > LN_MAX_N || C < 1 || C > LN_MAX_C) return LN_ERR_SHAPE;
@@ -177,7 +200,47 @@ void occ_store(const void *fn, int dev, int threads, size_t smem, int occ) {
     g_occ[OccKey{fn, dev, threads, smem}] = occ;
 }
 
+cudaError_t raise_smem_limit(const void *fn, int dev, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;   // within every kernel's default limit
+    std::lock_guard<std::mutex> lk(g_smem_mu);
+    size_t &limit = g_smem_limit[FnDev{fn, dev}];
+    if (limit >= smem) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+        note_cuda_error(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+        return e;
+    }
+    limit = smem;
+    return cudaSuccess;
+}
+
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int note_cuda_error(cudaError_t e, const char *call) {
+    t_last_error.code = e;
+    t_last_error.call = call;
+    return LN_ERR_CUDA;
+}
+
+cudaError_t workspace_pool(int dev, cudaMemPool_t *pool, uint64_t *limit) {
+    DeviceState &d = g_dev[dev];   // dev was validated by device_state
+    std::call_once(d.pool_once, [&]() {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaError_t e = cudaMemPoolCreate(&d.pool, &props);
+        if (e == cudaSuccess) {
+            uint64_t keep = UINT64_MAX;
+            e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        d.pool_error = e;
+    });
+    *pool = d.pool;
+    *limit = d.workspace_limit.load(std::memory_order_relaxed);
+    return d.pool_error;
+}
 
 // The backward behind ln_backward, ln_backward_ex and ln_backward_noalloc
 // (scratch != nullptr: partial sums in that array instead of the pool).
@@ -199,7 +262,7 @@ int backward_entry(void *dinp, float *dweight, float *dbias, const void *dout,
         if (acc_params) return LN_OK;   // nothing to add
         cudaError_t e = cudaMemsetAsync(dweight, 0, size_t(C) * sizeof(float), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(dbias, 0, size_t(C) * sizeof(float), s);
-        return status_of(e);
+        return e == cudaSuccess ? LN_OK : note_cuda_error(e, "cudaMemsetAsync");
     }
     if (!dinp || !dout || !inp || !weight) return LN_ERR_NULL;
     if (!recompute && (!mean || !rstd)) return LN_ERR_NULL;
@@ -215,7 +278,7 @@ int backward_entry(void *dinp, float *dweight, float *dbias, const void *dout,
     const BwdArgs a{dinp,          dweight,   dbias,    dout,     inp,
                     weight,        mean,      rstd,     N,        (int)C,
                     1.0f / float(C), eps,     acc_params, s,      dev,
-                    ds->sms,       ds->pool,  scratch,  scratch_floats, ds->status};
+                    ds->sms,       scratch,   scratch_floats, ds->status};
     const int mode = ((flags & LN_BWD_ACCUMULATE_DINP) ? lnk::kBwdAccumulate : 0) |
                      (recompute ? lnk::kBwdRecompute : 0);
     switch (dtype) {
@@ -282,14 +345,30 @@ int ln_device_status(unsigned int *bits, int clear) {
     int dev = 0;
     DeviceState *ds = nullptr;
     if (int st = current_device(&dev, &ds)) return st;
-    if (cudaMemcpy(bits, ds->status, sizeof(unsigned int), cudaMemcpyDeviceToHost) !=
-        cudaSuccess)
-        return LN_ERR_CUDA;
-    if (clear && cudaMemset(ds->status, 0, sizeof(unsigned int)) != cudaSuccess)
-        return LN_ERR_CUDA;
+    cudaError_t e = cudaMemcpy(bits, ds->status, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return lnh::note_cuda_error(e, "cudaMemcpy (device status word)");
+    if (clear && (e = cudaMemset(ds->status, 0, sizeof(unsigned int))) != cudaSuccess)
+        return lnh::note_cuda_error(e, "cudaMemset (device status word)");
     return LN_OK;
 }
 
-int ln_version(void) { return 2; }
+int ln_set_workspace_limit(int64_t bytes) {
+    if (bytes < 0) return LN_ERR_SHAPE;
+    int dev = 0;
+    DeviceState *ds = nullptr;
+    if (int st = current_device(&dev, &ds)) return st;
+    ds->workspace_limit.store(uint64_t(bytes), std::memory_order_relaxed);
+    return LN_OK;
+}
+
+const char *ln_last_cuda_error(void) {
+    const LastCudaError &l = t_last_error;
+    if (l.code == cudaSuccess) return "no CUDA error recorded on this thread";
+    snprintf(t_last_error_text, sizeof t_last_error_text, "%s (%d: %s) in %s",
+             cudaGetErrorName(l.code), int(l.code), cudaGetErrorString(l.code), l.call);
+    return t_last_error_text;
+}
+
+int ln_version(void) { return 3; }
 
 }  // extern "C"

@@ -13,11 +13,11 @@
 //
 // Workspace.  The backward needs G * 2C fp32 partial sums (G = its grid).
 // They are drawn stream-ordered from a memory pool that the library creates
-// once per device (release threshold: never), and handed back on the same
-// stream right after the finalise kernel, so calls on different streams never
-// share a buffer and steady-state calls reuse pool memory without a
-// cudaMalloc; or, for ln_backward_noalloc, they live in a static array whose
-// size caps G.
+// on the first pooled call on a device (release threshold: never), and handed
+// back on the same stream right after the finalise kernel, so calls on
+// different streams never share a buffer and steady-state calls reuse pool
+// memory without a cudaMalloc; or, for ln_backward_noalloc, they live in a
+// static array whose size caps G (that path never creates the pool).
 #pragma once
 
 #include "ln_host.cuh"
@@ -181,7 +181,12 @@ int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule
     float *partial = a.scratch;
     if (!partial) {
         const size_t ws_bytes = size_t(G) * 2 * size_t(a.C) * sizeof(float);
-        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), ws_bytes, a.pool,
+        cudaMemPool_t pool = nullptr;
+        uint64_t limit = 0;
+        const cudaError_t ep = workspace_pool(a.dev, &pool, &limit);
+        if (ep != cudaSuccess) return note_cuda_error(ep, "cudaMemPoolCreate (workspace pool)");
+        if (limit != 0 && ws_bytes > limit) return LN_ERR_WORKSPACE;
+        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), ws_bytes, pool,
                                     a.stream) != cudaSuccess) {
             cudaGetLastError();   // clear the non-sticky allocation error
             return LN_ERR_WORKSPACE;
@@ -207,7 +212,10 @@ int bwd_run(const BwdArgs &a, K kern, int threads, size_t smem, int rows_granule
     }
     if (!a.scratch) {
         const cudaError_t ef = cudaFreeAsync(partial, a.stream);
-        if (e == cudaSuccess) e = ef;
+        if (e == cudaSuccess && ef != cudaSuccess) {
+            note_cuda_error(ef, "cudaFreeAsync");
+            e = ef;
+        }
     }
     return status_of(e);
 }

@@ -17,7 +17,21 @@ namespace lnh {
 // ---- defined in ln_api.cu
 bool occ_find(const void *fn, int dev, int threads, size_t smem, int *occ);
 void occ_store(const void *fn, int dev, int threads, size_t smem, int occ);
+// Makes the kernel's dynamic shared-memory limit on `dev` (the current
+// device) at least `smem`.  The limit is one value per kernel and device, so
+// it only ever grows: a call with a smaller size leaves the larger limit of
+// an earlier call in place.
+cudaError_t raise_smem_limit(const void *fn, int dev, size_t smem);
 void count_launches(uint64_t n);
+// Records, for the calling host thread, the CUDA error behind the
+// LN_ERR_CUDA the library is about to return and the call that raised it
+// (read back with ln_last_cuda_error); returns LN_ERR_CUDA.
+int note_cuda_error(cudaError_t e, const char *call);
+// The stream-ordered pool that the pooled backward draws its partial sums
+// from on `dev` (created on the first call for that device, with it
+// current), and the per-call workspace cap set by ln_set_workspace_limit
+// (0: none).
+cudaError_t workspace_pool(int dev, cudaMemPool_t *pool, uint64_t *limit);
 // Validation and dispatch of every backward entry point; scratch != nullptr
 // keeps the partial sums in that device array (scratch_floats floats)
 // instead of drawing them from the pool.
@@ -30,24 +44,32 @@ constexpr size_t kMaxWorkspaceBytes = size_t(256) << 20;
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Status of a CUDA result whose failure the failing step has already noted
+// (launch, blocks_per_sm and raise_smem_limit note their own errors).
 inline int status_of(cudaError_t e) { return e == cudaSuccess ? LN_OK : LN_ERR_CUDA; }
 
 // Resident blocks per SM of `kernel` at this block size and dynamic shared
-// memory (computed once per kernel, device and size; also raises the
-// kernel's dynamic shared-memory limit on that device when needed).
+// memory (computed once per kernel, device and size).  Every call, cached or
+// not, first makes sure the kernel's dynamic shared-memory limit on that
+// device admits `smem`, since a launch is checked against the limit in force
+// when it is made, not against the one of the call that filled the cache.
 template <typename K>
 cudaError_t blocks_per_sm(K kernel, int dev, int threads, size_t smem, int *occ) {
     const void *fn = reinterpret_cast<const void *>(kernel);
-    if (occ_find(fn, dev, threads, smem, occ)) return cudaSuccess;
-    cudaError_t e = cudaSuccess;
-    if (smem > 48 * 1024)
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-    int n = 0;
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    cudaError_t e = raise_smem_limit(fn, dev, smem);
     if (e != cudaSuccess) return e;
-    if (n < 1) return cudaErrorInvalidConfiguration;
+    if (occ_find(fn, dev, threads, smem, occ)) return cudaSuccess;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    if (e != cudaSuccess) {
+        note_cuda_error(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+        return e;
+    }
+    if (n < 1) {
+        note_cuda_error(cudaErrorInvalidConfiguration,
+                        "cudaOccupancyMaxActiveBlocksPerMultiprocessor (no block fits an SM)");
+        return cudaErrorInvalidConfiguration;
+    }
     occ_store(fn, dev, threads, smem, n);
     *occ = n;
     return cudaSuccess;
@@ -71,7 +93,10 @@ cudaError_t launch(K kernel, int grid, int threads, size_t smem, cudaStream_t st
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
-    if (e == cudaSuccess) count_launches(1);
+    if (e == cudaSuccess)
+        count_launches(1);
+    else
+        note_cuda_error(e, "cudaLaunchKernelEx");
     return e;
 }
 
@@ -97,7 +122,8 @@ struct FwdArgs {
 };
 
 // Backward call.  The per-block partial sums come from `scratch` (capacity
-// scratch_floats, no allocation) when it is set, else from `pool`.
+// scratch_floats, no allocation) when it is set, else from the device's
+// workspace pool (workspace_pool).
 struct BwdArgs {
     void *dinp;
     float *dweight;
@@ -115,7 +141,6 @@ struct BwdArgs {
     cudaStream_t stream;
     int dev;
     int sms;
-    cudaMemPool_t pool;
     float *scratch;
     int64_t scratch_floats;
     unsigned int *status;

@@ -20,11 +20,17 @@
 //     the variance from the deviations held in registers: a plain fp32 sum of
 //     x, or E[x^2] - E[x]^2, loses the variance of rows such as 100 + 0.01 z;
 //   * weight and bias are staged once per block in shared memory;
-//   * the column sums of the backward are deterministic: each block owns a
-//     fixed, contiguous range of rows, accumulates its columns in registers,
-//     combines its row groups in a fixed order and writes one partial row;
-//     a second kernel sums the partial rows in a fixed order.  No float
-//     atomics anywhere.
+//   * the column sums of the backward are deterministic: each block of the
+//     row kernel owns a fixed set of rows (register-resident and scalar
+//     kernels: a contiguous range; TMA ring: tiles dealt round-robin over
+//     the blocks), accumulates its columns in registers, combines its warps
+//     in a fixed order and writes one partial row; a second kernel sums the
+//     G partial rows in a fixed order.  Which rows a block owns depends only
+//     on N, C and the grid G, and G = SMs x resident blocks per SM (capped
+//     by the rows, and by the static array for ln_backward_noalloc), so the
+//     bits of dweight/dbias are fixed for a given device model and call, but
+//     may differ between devices with different SM counts.  No float atomics
+//     anywhere.
 // No kernel waits on another block or on a flag: the only cross-kernel
 // dependency is programmatic dependent launch (griddepcontrol), resolved by
 // the hardware when the producing grid completes.
@@ -39,6 +45,11 @@ namespace lnk {
 
 using bf16 = __nv_bfloat16;
 using f16 = __half;
+
+// The dynamic shared memory of every kernel in this library, declared once
+// with one alignment (128 bytes: TMA bulk-copy destinations and mbarriers are
+// carved from it at 128-byte offsets).
+extern __shared__ __align__(128) unsigned char ln_dyn_smem[];
 
 // Elements per 16-byte vector.
 template <typename T> struct Vec;
@@ -378,7 +389,7 @@ ln_fwd_vec_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restri
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
-    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char *smem = ln_dyn_smem;
     const int nvec = C / E;
     float *s_w = reinterpret_cast<float *>(smem);
     float *s_b = s_w + C;
@@ -510,7 +521,7 @@ ln_bwd_vec_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
     constexpr int TPR = 32 * W;
-    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char *smem = ln_dyn_smem;
     const int nvec = C / E;
     float *s_w = reinterpret_cast<float *>(smem);
     float *s_acc = s_w + C;                                   // [GROUPS/2][2C]

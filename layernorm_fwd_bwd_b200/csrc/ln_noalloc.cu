@@ -66,9 +66,12 @@ extern "C" int ln_backward_noalloc(void *dinp, float *dweight, float *dbias,
     if (dtype != LN_F32 && dtype != LN_BF16 && dtype != LN_F16) return LN_ERR_DTYPE;
     if (C > LN_NOALLOC_MAX_C) return LN_ERR_SCRATCH;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LN_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return lnh::note_cuda_error(e, "cudaGetDevice");
     ScratchDevice *sd = nullptr;
-    if (scratch_device(dev, &sd) != cudaSuccess) return LN_ERR_CUDA;
+    e = scratch_device(dev, &sd);
+    if (e != cudaSuccess)
+        return lnh::note_cuda_error(e, "cudaGetSymbolAddress (no-alloc scratch array)");
     return lnh::backward_entry(dinp, dweight, dbias, dout, inp, weight, mean, rstd, N, C, 0.f,
                                dtype, 0u, stream, sd->scratch, kScratchFloats);
 }

@@ -83,7 +83,7 @@ ln_fwd_tile_kernel(T *__restrict__ out, float *__restrict__ mean, float *__restr
     constexpr int P = E / 2;
     constexpr int RT = NW / W;                                // rows per tile
     constexpr int TPR = 32 * W;
-    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char *smem = ln_dyn_smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);      // [0]: params, [1+t]: tile t
     const uint32_t row_bytes = uint32_t(C) * sizeof(T);
     unsigned char *s_par = smem + 128;                         // weight then bias, raw

@@ -225,7 +225,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     constexpr int P = E / 2;
     constexpr int RT = NC / W;                               // rows per tile
     constexpr int TPR = 32 * W;                              // threads per row
-    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char *smem = ln_dyn_smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + S;
     float *s_w = reinterpret_cast<float *>(smem + 128);      // weight as fp32

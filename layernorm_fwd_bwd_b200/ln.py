@@ -68,12 +68,22 @@ _lib.ln_version.restype = _int
 _lib.ln_version.argtypes = []
 _lib.ln_device_status.restype = _int
 _lib.ln_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), _int]
+_lib.ln_set_workspace_limit.restype = _int
+_lib.ln_set_workspace_limit.argtypes = [_i64]
+_lib.ln_last_cuda_error.restype = ctypes.c_char_p
+_lib.ln_last_cuda_error.argtypes = []
 
 
 class LNError(RuntimeError):
+    """A non-LN_OK status; for LN_ERR_CUDA the message also names the CUDA
+    error and the runtime call that raised it."""
+
     def __init__(self, status: int):
         self.status = status
-        super().__init__(ln_status_string(status))
+        msg = ln_status_string(status)
+        if status == LN_ERR_CUDA:
+            msg += f" [{last_cuda_error()}]"
+        super().__init__(msg)
 
 
 def library_path() -> str:
@@ -90,6 +100,17 @@ def launch_count() -> int:
 
 def version() -> int:
     return int(_lib.ln_version())
+
+
+def last_cuda_error() -> str:
+    """The CUDA error behind this thread's most recent LN_ERR_CUDA."""
+    return _lib.ln_last_cuda_error().decode()
+
+
+def set_workspace_limit(nbytes: int) -> None:
+    """Cap the pooled backward's workspace per call on the current device
+    (0: no cap); a call needing more fails with LN_ERR_WORKSPACE."""
+    _check(_lib.ln_set_workspace_limit(int(nbytes)))
 
 
 def device_status(clear: bool = False) -> int:

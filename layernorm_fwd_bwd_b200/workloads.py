@@ -46,8 +46,10 @@ dweight and dbias, fp32 N(0,1).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -197,8 +199,11 @@ def _rows_block(w: Workload, rows: np.ndarray, stream: int, mu: float,
     return mu + sigma * normals(w.seed, stream, idx.reshape(-1)).reshape(len(rows), C)
 
 
-def generate(w: Workload, rows=None, chunk_rows: int = 8192) -> Batch:
-    """Draw the workload's inputs for ``rows`` (all rows when None)."""
+def generate(w: Workload, rows=None, chunk_rows: int = 8192, workers: int = 0) -> Batch:
+    """Draw the workload's inputs for ``rows`` (all rows when None).  Chunks
+    of rows are drawn on ``workers`` threads (0: up to 8, by the host's core
+    count); the counter-based generator makes every element independent of
+    the chunking and of the thread that draws it."""
     rows = np.arange(w.N, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
     if rows.size and (rows.min() < 0 or rows.max() >= w.N):
         raise ValueError("row index out of range")
@@ -208,7 +213,8 @@ def generate(w: Workload, rows=None, chunk_rows: int = 8192) -> Batch:
     store = np.float32 if w.dtype == F32 else np.uint16
     inp = np.empty((rows.size, w.C), store)
     dout = np.empty((rows.size, w.C), store)
-    for a in range(0, rows.size, chunk_rows):
+
+    def chunk(a):
         rr = rows[a:a + chunk_rows]
         x = _rows_block(w, rr, S_INP, w.inp_mu, w.inp_sigma)
         if w.const_row_period:
@@ -219,6 +225,15 @@ def generate(w: Workload, rows=None, chunk_rows: int = 8192) -> Batch:
         inp[a:a + rr.size] = to_storage(x, w.dtype)
         dout[a:a + rr.size] = to_storage(
             _rows_block(w, rr, S_DOUT, 0.0, w.dout_sigma), w.dtype)
+
+    starts = range(0, rows.size, chunk_rows)
+    n = workers or min(8, os.cpu_count() or 1)
+    if n > 1 and len(starts) > 1:
+        with concurrent.futures.ThreadPoolExecutor(n) as ex:
+            list(ex.map(chunk, starts))
+    else:
+        for a in starts:
+            chunk(a)
     return Batch(w, rows, inp, weight, bias, dout)
 
 

@@ -79,3 +79,14 @@ def test_no_kernel_spills_heavily(kernels):
     heavy = {n: k for n, k in kernels.items()
              if max(k["spill_st"], k["spill_ld"], k["stack"]) > MAX_SPILL_BYTES}
     assert not heavy, heavy
+
+
+def test_no_compiler_warnings(kernels):
+    """Every object compiles without a compiler warning (for example #1886-D,
+    which nvcc gives when two kernels declare the dynamic shared array with
+    different alignments)."""
+    from layernorm_fwd_bwd_b200 import build
+    for obj in build.objects():
+        text = open(build.ptxas_report(obj)).read()
+        warnings = [line for line in text.splitlines() if re.search(r"\bwarning\b", line)]
+        assert not warnings, f"{os.path.basename(obj)}: {warnings[:3]}"

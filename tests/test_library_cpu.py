@@ -51,7 +51,7 @@ def test_status_strings(lib):
         assert lib.ln_status_string(code).startswith(name)
         assert getattr(lib, name) == code
     assert lib.ln_status_string(99) == "unknown ln_status"
-    assert lib.version() == 2
+    assert lib.version() == 3
 
 
 def test_host_validation_without_gpu(lib):
@@ -334,3 +334,54 @@ def test_header_compiles_as_cpp():
     subprocess.run(["g++", "-std=c++11", "-Wall", "-Werror", "-pedantic", "-I",
                     os.path.join(ROOT, "include"), "-x", "c++", "-", "-fsyntax-only"],
                    input=src, text=True, check=True)
+
+
+def test_workspace_limit_and_last_cuda_error_on_host(lib):
+    """ln_set_workspace_limit refuses a negative cap before touching CUDA;
+    without a usable device it returns LN_ERR_CUDA, and ln_last_cuda_error
+    then names the runtime call that failed."""
+    import torch
+    assert lib._lib.ln_set_workspace_limit(-1) == lib.LN_ERR_SHAPE
+    assert isinstance(lib.last_cuda_error(), str) and lib.last_cuda_error()
+    if torch.cuda.is_available():
+        pytest.skip("a device is present: the failing path is not reachable here")
+    assert lib._lib.ln_set_workspace_limit(0) == lib.LN_ERR_CUDA
+    text = lib.last_cuda_error()
+    assert "cudaGetDevice" in text and text.startswith("cuda"), text
+    with pytest.raises(lib.LNError) as e:
+        lib.set_workspace_limit(0)
+    assert "cudaGetDevice" in str(e.value)
+
+
+def _code(path):
+    """C++ source with comments and string literals removed."""
+    text = open(path).read()
+    text = re.sub(r"//[^\n]*", "", text)
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.sub(r'"(?:\\.|[^"\\])*"', '""', text)
+
+
+def test_only_the_pooled_backward_creates_the_pool():
+    """ln_backward_noalloc must not create the library's memory pool: the
+    pool is created in one function (workspace_pool), which is reached only
+    from the branch of the backward that has no caller-provided scratch."""
+    csrc = os.path.join(ROOT, "layernorm_fwd_bwd_b200", "csrc")
+    creators, callers = [], []
+    for f in sorted(os.listdir(csrc)):
+        code = _code(os.path.join(csrc, f))
+        if "cudaMemPoolCreate" in code:
+            creators.append(f)
+        for m in re.finditer(r"\bworkspace_pool\s*\(", code):
+            callers.append((f, code[:m.start()]))
+    assert creators == ["ln_api.cu"]
+    api = _code(os.path.join(csrc, "ln_api.cu"))
+    body = api[api.index("cudaError_t workspace_pool("):]
+    body = body[:body.index("\n}\n")]
+    assert "cudaMemPoolCreate" in body
+    assert api.count("cudaMemPoolCreate") == 1
+    uses = [(f, pre) for f, pre in callers
+            if not re.search(r"cudaError_t\s+$", pre)]   # skip declarations/definition
+    assert [f for f, _ in uses] == ["ln_dispatch.cuh"], uses
+    pre = uses[0][1]
+    branch = pre[pre.rindex("float *partial = a.scratch;"):]
+    assert re.search(r"if\s*\(\s*!\s*partial\s*\)\s*\{", branch), branch[-300:]

@@ -289,6 +289,69 @@ def test_deterministic(lib, name):
             assert torch.equal(bits(a), bits(b))
 
 
+# (dtype, N, C of the first and third call, C of the second): one kernel
+# instantiation each, whose dynamic shared memory grows with C.  The second C
+# appears in no other test, so its first call always sets up that kernel at a
+# smaller size after the larger one.
+SHRINK_GROW = [("bf16", 64, 16384, 15992),   # register-resident forward, 16 warps per row
+               ("bf16", 4096, 768, 648),     # tile forward, one-warp ring backward
+               ("f32", 2048, 2560, 2440),    # fp32 ring backward, shared rows
+               ("bf16", 1024, 4096, 3976)]   # two-warp tile forward, wide backward
+
+
+@pytest.mark.parametrize("dtype,N,C_big,C_small", SHRINK_GROW)
+def test_shapes_shrinking_then_growing(lib, dtype, N, C_big, C_small):
+    """A kernel's dynamic shared-memory limit is one value per kernel and
+    device: a call at a smaller C must not leave a limit that a later call
+    at the larger C, whose set-up was cached, launches above.  Every call
+    returns LN_OK and matches the oracle."""
+    for C in (C_big, C_small, C_big):
+        batch = wl.custom(dtype, N, C, seed=3000 + C)
+        label = f"{dtype} {N}x{C}"
+        dev, _, ref_stats, _ = _forward_parity(lib, batch, label, scaled=True)
+        _backward_parity(lib, batch, dev, label, ref_stats, scaled=True)
+
+
+def test_workspace_refusal_launches_nothing(lib):
+    """LN_ERR_WORKSPACE: a backward whose partial sums exceed the device's
+    workspace cap is refused before any launch, leaves the outputs and the
+    CUDA context untouched, and the next call within the cap succeeds."""
+    N, C = 4096, 768
+    batch = wl.custom("bf16", N, C, seed=31)
+    inp, wt, bs, dout = gu.batch_to_device(batch)
+    _, mean, rstd = gu.forward(lib, inp, wt, bs, N, C, batch.eps, "bf16")
+    want = gu.backward(lib, dout, inp, wt, mean, rstd, N, C, "bf16")
+    torch.cuda.synchronize()
+    dinp = gu.nan_tensor((N, C), torch.bfloat16)
+    dw = gu.nan_tensor((C,), torch.float32)
+    db = gu.nan_tensor((C,), torch.float32)
+    try:
+        lib.set_workspace_limit(2 * C * 4 - 1)        # less than one block's partial row
+        before = lib.launch_count()
+        for call in (lambda: lib.ln_backward(dinp, dw, db, dout, inp, wt, mean, rstd, N, C,
+                                             lib.LN_BF16),
+                     lambda: lib.ln_backward_ex(dinp, dw, db, dout, inp, wt, None, None, N, C,
+                                                batch.eps, lib.LN_BF16,
+                                                lib.LN_BWD_RECOMPUTE_STATS)):
+            with pytest.raises(lib.LNError) as e:
+                call()
+            assert e.value.status == lib.LN_ERR_WORKSPACE
+        assert lib.launch_count() == before
+        torch.cuda.synchronize()                          # no error left behind
+        assert bool(torch.isnan(dinp.float()).all()) and bool(torch.isnan(dw).all())
+        # the allocation-free entry point does not draw from the pool
+        lib.ln_backward_noalloc(dinp, dw, db, dout, inp, wt, mean, rstd, N, C, lib.LN_BF16)
+        torch.cuda.synchronize()
+        assert lib.launch_count() == before + 2
+    finally:
+        lib.set_workspace_limit(0)
+    got = gu.backward(lib, dout, inp, wt, mean, rstd, N, C, "bf16")
+    torch.cuda.synchronize()
+    for g, r in zip(got, want):
+        assert bool((gu.bits(g) == gu.bits(r)).all())
+    assert lib.device_status() == 0
+
+
 def test_empty_batch(lib):
     C = 64
     w = torch.ones(C, device="cuda")

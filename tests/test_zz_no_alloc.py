@@ -5,8 +5,9 @@ partial sums in a static device array inside the library instead of the
 stream-ordered pool ln_backward uses.
 
 Checked through the C ABI against ln_backward on the same inputs, within the
-tolerances the other parity tests use, on two calls in a row with different
-inputs (the static array keeps the first call's contents, so the second call
+tolerances the other parity tests use, on two calls in a row: with different
+inputs of one shape, and with a second shape on fewer blocks or another row
+width (the static array keeps the first call's contents, so the second call
 shows that nothing stale leaks in).  This file is collected last so that a run
 stopping at its first failure has already run every other test."""
 import pytest
@@ -51,6 +52,35 @@ def _noalloc(lib, dout, inp, wt, mean, rstd, N, C, dtype):
 def test_noalloc_matches_ln_backward_twice(lib, dtype, N, C):
     for call, seed in enumerate((101, 202)):
         batch = wl.custom(dtype, N, C, seed=seed + C)
+        dev = gu.batch_to_device(batch)
+        inp, wt, _, dout = dev
+        mean, rstd = _stats(lib, batch, dev)
+        want = gu.backward(lib, dout, inp, wt, mean, rstd, N, C, dtype)
+        got = _noalloc(lib, dout, inp, wt, mean, rstd, N, C, dtype)
+        torch.cuda.synchronize()
+        for name, kind, g, r in zip(("dinp", "dweight", "dbias"),
+                                    ("act_bwd", "param_grad", "param_grad"), got, want):
+            assert not bool(torch.isnan(g.float()).any()), f"call {call}: {name} not written"
+            tol.check(f"call {call} {dtype} {N}x{C} {name}", gu.to_f64(g), gu.to_f64(r),
+                      dtype, kind)
+
+
+# Two calls in a row with different shapes, the second on fewer blocks or a
+# different row width than the first: the array still holds the first call's
+# partial rows (laid out for its C), so a finalise that read a row its own
+# call did not write would change dweight or dbias.
+SEQUENCES = [
+    (("bf16", 300, 16384), ("bf16", 64, 768)),     # 32 capped blocks, then 5 blocks
+    (("f32", 1000, 1600), ("bf16", 4096, 768)),
+    (("bf16", 4096, 768), ("bf16", 20, 1024)),
+    (("f16", 2048, 1600), ("f32", 513, 7)),        # then the scalar path
+]
+
+
+@pytest.mark.parametrize("first,second", SEQUENCES)
+def test_noalloc_after_a_different_shape(lib, first, second):
+    for call, (dtype, N, C) in enumerate((first, second)):
+        batch = wl.custom(dtype, N, C, seed=707 + 13 * call + C)
         dev = gu.batch_to_device(batch)
         inp, wt, _, dout = dev
         mean, rstd = _stats(lib, batch, dev)
