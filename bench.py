@@ -55,7 +55,7 @@ EVERY = 64          # per-call events on one timed step in EVERY
 # traffic figure stays valid while these are unchanged)
 KERNEL_SOURCES = [os.path.join(ROOT, "layernorm_fwd_bwd_b200", "csrc", f)
                   for f in ("ln_kernels.cuh", "ln_select.cuh", "ln_tma.cuh", "ln_tile.cuh",
-                            "ln_dispatch.cuh", "ln_host.cuh")]
+                            "ln_split.cuh", "ln_dispatch.cuh", "ln_host.cuh")]
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "ln_backward_gpt2_124m_bf16.md")
 
 
@@ -76,6 +76,9 @@ def parse_args():
                    help="skip timing ln_forward_residual, ln_backward_ex and fp16")
     p.add_argument("--no-workloads", action="store_true",
                    help="skip timing forward and backward on every workload")
+    p.add_argument("--no-loops", action="store_true",
+                   help="time the K steps only: no back-to-back call loops, e2e, variants "
+                        "or workloads (short runs under a profiler)")
     p.add_argument("--sets", type=int, default=SETS,
                    help="rotating buffer sets (>= 2 so a step's backward never "
                         "reads what its forward just read)")
@@ -340,8 +343,12 @@ def run_ours(args, world: int, rank: int, local: int):
     total_ms = max_over_ranks(total_ms, dev)
 
     # each call on its own, back to back (events around the loop only)
-    fwd_loop_us = call_loop_us(torch, stream, lambda i: check(fwd(*fargs[i % nsets])))
-    bwd_loop_us = call_loop_us(torch, stream, lambda i: check(bwd(*bargs[i % nsets])))
+    if args.no_loops:
+        args.no_e2e = args.no_variants = args.no_workloads = True
+        fwd_loop_us, bwd_loop_us = fwd_ms * 1e3, bwd_ms * 1e3
+    else:
+        fwd_loop_us = call_loop_us(torch, stream, lambda i: check(fwd(*fargs[i % nsets])))
+        bwd_loop_us = call_loop_us(torch, stream, lambda i: check(bwd(*bargs[i % nsets])))
 
     # end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else run_e2e(args, torch, ln, stream, dev, h_inp, h_dout,
@@ -367,6 +374,8 @@ def run_ours(args, world: int, rank: int, local: int):
     peak, peak_kind = hbm_peak()
     bwd_gbs = bb / (bwd_loop_us / 1e6) / 1e9
     fwd_gbs = fb / (fwd_loop_us / 1e6) / 1e9
+    loop_timing = (f"{LOOP_CALLS} back-to-back calls over the rotating sets" if not args.no_loops
+                   else "events around each call of the sampled timed steps (--no-loops)")
     clocks = None
     if sampler:
         clocks = sampler.summary(t0, t_loops)
@@ -387,10 +396,10 @@ def run_ours(args, world: int, rank: int, local: int):
         "pct_hbm_measured": round(value / world / peak * 100, 2) if peak_kind == "measured" else None,
         "pct_hbm_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS * 100, 2),
         "fwd": {"us": round(fwd_loop_us, 3), "GB_s": round(fwd_gbs, 1), "bytes": fb,
-                "timing": f"{LOOP_CALLS} back-to-back calls over the rotating sets",
+                "timing": loop_timing,
                 "us_sampled_in_step": round(fwd_ms * 1e3, 3)},
         "bwd": {"us": round(bwd_loop_us, 3), "GB_s": round(bwd_gbs, 1), "bytes": bb,
-                "timing": f"{LOOP_CALLS} back-to-back calls over the rotating sets",
+                "timing": loop_timing,
                 "us_sampled_in_step": round(bwd_ms * 1e3, 3)},
         "per_call_sampling": f"events around each call on 1 timed step in {EVERY} "
                              f"({len(events)} steps); an event between two launches "

@@ -230,6 +230,16 @@ struct BwdVec {
                                    32 * W * GROUPS, lnk::bwd_vec_smem<W, GROUPS>(a.C),
                                    GROUPS, 1);
     }
+    template <int VR, int VC>
+    void split() {
+        constexpr int NS = lnk::BwdRingArrays<MODE>::value;
+        constexpr int NR = lnk::kSplitRowWarps;
+        constexpr int S_MAX = lnk::kSplitMaxStages;
+        const int S = std::min(lnk::split_stages<T, NR, NS>(a.C, lnk::kMaxSmemPerBlock), S_MAX);
+        status = bwd_run<T, true>(
+            a, lnk::ln_bwd_split_kernel<T, VR, VC, NR, lnk::kSplitColWarps, MODE>,
+            32 * (NR + lnk::kSplitColWarps + 1), lnk::split_smem<T, NR, NS>(a.C, S), NR, NR);
+    }
     template <int V, int W>
     void ring() {
         constexpr int NS = lnk::BwdRingArrays<MODE>::value;

@@ -7,14 +7,17 @@
 // warps per row; wider rows take the persistent register-resident kernel
 // with W = 4, 8 or 16 warps per row and 4 vectors per thread.
 // Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
-// persistent TMA-ring kernel (ln_tma.cuh) on one warp per row, wider rows the
-// ring with W = 2..4 warps per row; rows wider than that take the
-// register-resident kernel (W = 4..16 warps per row, 4 vectors per thread).
+// persistent TMA-ring kernel (ln_tma.cuh) on one warp per row; 16-bit rows of
+// 7..8 vectors per lane (plain and accumulating) the split ring of row and
+// column warps (ln_split.cuh); other wider rows the ring with W = 2..4 warps
+// per row; rows wider than that take the register-resident kernel (W =
+// 4..16 warps per row, 4 vectors per thread).
 // Rows wider than the widest variant, and any misaligned call, take the
 // scalar kernels.
 #pragma once
 
 #include "ln_kernels.cuh"
+#include "ln_split.cuh"
 #include "ln_tile.cuh"
 #include "ln_tma.cuh"
 
@@ -156,8 +159,36 @@ template <int MODE> struct RingVmax<float, MODE> {
     static constexpr int one = kAcc ? 4 : 6, shared = kAcc ? 4 : 5;
 };
 
-// Calls visitor.template ring<V, W>(); false when rows are wider than 4 warps
-// cover.
+// Row warps (rows per tile) and column warps of the split backward
+// (ln_split.cuh), and the widest row it serves in 16-byte vectors per lane of
+// a row warp.  It takes 16-bit rows of LN_SPLIT_FROM_V .. kSplitMaxV vectors
+// per lane in the plain and dinp-accumulating backward; with
+// recomputed statistics (the column warps would need the row warps' results
+// first) those rows stay on the shared-row ring.  8 + 4 warps and the
+// producer: ptxas fits the layout in 128 registers without spilling (13 warps
+// x 32 x 128 of the SM's 65536), and 8-row stages of bf16 C = 1600 leave room
+// for a 4-deep ring.
+// Measured on B200 (bf16, back-to-back calls): C = 2048 26.7 us against 28.3
+// on the shared-row ring, C = 1600 40.0 against 39.6 (accumulating 43.6
+// against 45.2), C = 1280 33.1 against 27.7, C = 1024 46.2 against 41.6 (one
+// warp per row); so rows from 7 vectors per lane.
+#ifndef LN_SPLIT_FROM_V
+#define LN_SPLIT_FROM_V 7
+#endif
+constexpr int kSplitRowWarps = 8;
+constexpr int kSplitColWarps = 4;
+constexpr int kSplitMaxV = 8;
+template <typename T, int MODE> struct SplitServes {
+    static constexpr bool value = sizeof(T) == 2 && (MODE & kBwdRecompute) == 0;
+};
+// Column-warp vectors per lane for rows of 32 * VR vectors.
+template <int VR> struct SplitVc {
+    static constexpr int value =
+        ((32 * VR + kSplitColWarps - 1) / kSplitColWarps + 31) / 32;
+};
+
+// Calls visitor.template ring<V, W>() or visitor.template split<VR, VC>();
+// false when rows are wider than 4 warps of the ring cover.
 template <typename T, int MODE, typename Visitor>
 bool visit_bwd_ring(int nvec, Visitor &v) {
     constexpr int NS = BwdRingArrays<MODE>::value;
@@ -168,6 +199,18 @@ bool visit_bwd_ring(int nvec, Visitor &v) {
     static_assert(bwd_ring_smem_max<T, VS, 3, NS>() <= kMaxSmemPerBlock, "ring fits");
     static_assert(bwd_ring_smem_max<T, VS, 4, NS>() <= kMaxSmemPerBlock, "ring fits");
     const int v1 = (nvec + 31) / 32;
+    if constexpr (SplitServes<T, MODE>::value) {
+        if (v1 >= LN_SPLIT_FROM_V && v1 <= kSplitMaxV) {
+            switch (v1) {
+                case 4: v.template split<4, SplitVc<4>::value>(); return true;
+                case 5: v.template split<5, SplitVc<5>::value>(); return true;
+                case 6: v.template split<6, SplitVc<6>::value>(); return true;
+                case 7: v.template split<7, SplitVc<7>::value>(); return true;
+                case 8: v.template split<8, SplitVc<8>::value>(); return true;
+                default: break;
+            }
+        }
+    }
     switch (v1) {
         case 1: v.template ring<1, 1>(); return true;
         case 2: v.template ring<2, 1>(); return true;

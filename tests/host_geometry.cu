@@ -15,7 +15,9 @@
 //     also with the one-tile and register-resident fallbacks the launcher
 //     may take;
 //   - the ring has 2..8 stages (its 128-byte barrier area holds 16) and
-//     whole row groups of consumer warps;
+//     whole row groups of consumer warps; the split ring (row and column
+//     warps) serves exactly the 16-bit rows of its range, its column warps
+//     cover their slices and its 2..8 stages fit;
 //   - every bulk copy is a whole number of 16-byte units, and the bytes one
 //     mbarrier phase expects (all the copies that complete on it) stay below
 //     the 2^20 limit of an mbarrier's transaction count.
@@ -141,13 +143,36 @@ struct BwdChoice {
             check(V == cdiv(nvec, 32) && V <= ONE,
                   ctx() + "one-warp ring rows take the fewest vectors per lane");
         else
-            check(V == VS && W == cdiv(nvec, 32 * VS) && nvec > 32 * ONE,
+            check(V == VS && W == cdiv(nvec, 32 * VS) && nvec > 32 * ONE &&
+                      (!lnk::SplitServes<T, MODE>::value || cdiv(nvec, 32) < LN_SPLIT_FROM_V ||
+                       nvec > 32 * lnk::kSplitMaxV),
                   ctx() + "shared ring rows: the fixed vectors per lane, the fewest warps, "
-                          "only past one warp's reach");
+                          "only past one warp's and the split kernel's reach");
+        if (lnk::SplitServes<T, MODE>::value)
+            check(cdiv(nvec, 32) < LN_SPLIT_FROM_V || cdiv(nvec, 32) > lnk::kSplitMaxV,
+                  ctx() + "rows the split kernel serves do not take the ring");
         check(S >= 2 && S <= 8, ctx() + "ring depth 2..8");
         check(NC % W == 0 && NC >= W, ctx() + "whole row groups of consumer warps");
         check(lnk::bwd_tma_smem<T, NC, S, W, NS>(C) <= kMax, ctx() + "ring shared memory fits");
         check_copies(ctx(), size_t(C) * sizeof(T), NC / W, NS);
+    }
+    template <int VR, int VC>
+    void split() {
+        const int C = nvec * E;
+        constexpr int NR = lnk::kSplitRowWarps, NCOL = lnk::kSplitColWarps;
+        const int S = lnk::split_stages<T, NR, NS>(C, kMax);
+        label = "split VR=" + num(VR) + " VC=" + num(VC) + " S=" + num(S);
+        check(lnk::SplitServes<T, MODE>::value, ctx() + "split rows: 16-bit, statistics read");
+        check(VR == cdiv(nvec, 32) && VR >= LN_SPLIT_FROM_V && VR <= lnk::kSplitMaxV,
+              ctx() + "split rows take the fewest vectors per row-warp lane, in its range");
+        check(32 * VC >= cdiv(nvec, NCOL) && 32 * (VC - 1) < cdiv(nvec, NCOL),
+              ctx() + "column warps cover their slices with the fewest vectors per lane");
+        check(S >= 2 && S <= lnk::kSplitMaxStages, ctx() + "split ring depth 2..8");
+        check(2 * lnk::kSplitMaxStages * 8 <= 128, ctx() + "split barriers fit in 128 bytes");
+        check(lnk::split_smem<T, NR, NS>(C, S) <= kMax, ctx() + "split shared memory fits");
+        check(lnk::split_ring_offset(C) % 128 == 0, ctx() + "split ring starts 128-aligned");
+        check(32 * (NR + NCOL + 1) <= 1024, ctx() + "split block size");
+        check_copies(ctx(), size_t(C) * sizeof(T), NR, NS);
     }
     template <int V, int W, int G>
     void run() {

@@ -112,6 +112,23 @@ def test_shape_sweep(lib, dtype, C, N):
     _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
 
 
+# Widths around and inside the split backward (16-bit rows of 7..8 vectors per
+# row-warp lane, row and column warps on one ring; narrower rows take the
+# rings next to it): column slices that end inside a warp and rings of 3 and 4
+# stages.  N = 7 is one partial tile; N = 5003 gives each block about four
+# tiles of 8 rows and a last tile of 3.
+SPLIT_C = [1032, 1184, 1192, 1416, 1536, 1760, 1784, 1800, 2040]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("C", SPLIT_C)
+@pytest.mark.parametrize("N", [7, 5003])
+def test_split_backward_widths(lib, dtype, C, N):
+    batch = wl.custom(dtype, N, C, seed=5000 + C + N, dout_sigma=0.02)
+    dev, _, ref_stats, _ = _forward_parity(lib, batch, f"{dtype} {N}x{C}", scaled=True)
+    _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_widest_row(lib, dtype):
     """C = LN_MAX_C (2^24 channels, 32 or 64 MB a row), two rows, every

@@ -142,6 +142,20 @@ def test_variant_sweep(lib, dtype, C, N):
         _backward_ex(lib, batch, extras, FLAG_SETS[fl], f"{label} {fl}", scaled=True)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("C", [1032, 1800, 2040])
+@pytest.mark.parametrize("N", [7, 5003])
+def test_split_accumulate_widths(lib, dtype, C, N):
+    """The split backward with three arrays per stage (dinp accumulated) on
+    partial and multi-tile blocks, and the recomputing backward at the same
+    widths (the shared-row ring)."""
+    batch = wl.custom(dtype, N, C, seed=6000 + C + N, dout_sigma=0.02)
+    extras = wl.generate_extras(batch.workload)
+    label = f"{dtype} {N}x{C}"
+    for fl in ("acc", "acc_params_only", "recompute"):
+        _backward_ex(lib, batch, extras, FLAG_SETS[fl], f"{label} {fl}", scaled=True)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("C", [768, 1600, 5])
 def test_variants_misaligned(lib, dtype, C):
