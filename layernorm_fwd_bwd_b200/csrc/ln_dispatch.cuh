@@ -235,10 +235,12 @@ struct BwdVec {
         constexpr int NS = lnk::BwdRingArrays<MODE>::value;
         constexpr int NR = lnk::kSplitRowWarps;
         constexpr int S_MAX = lnk::kSplitMaxStages;
-        const int S = std::min(lnk::split_stages<T, NR, NS>(a.C, lnk::kMaxSmemPerBlock), S_MAX);
-        status = bwd_run<T, true>(
-            a, lnk::ln_bwd_split_kernel<T, VR, VC, NR, lnk::kSplitColWarps, MODE>,
-            32 * (NR + lnk::kSplitColWarps + 1), lnk::split_smem<T, NR, NS>(a.C, S), NR, NR);
+        const int S =
+            std::min(lnk::split_stages<T, NR, NS>(a.C, lnk::kMaxSmemPerBlock), S_MAX);
+        constexpr int NCOL = lnk::SplitCols<VR>::value;
+        status = bwd_run<T, true>(a, lnk::ln_bwd_split_kernel<T, VR, VC, NR, NCOL, MODE>,
+                                  32 * (NR + NCOL + 1), lnk::split_smem<T, NR, NS>(a.C, S),
+                                  NR, NR);
     }
     template <int V, int W>
     void ring() {

@@ -159,32 +159,36 @@ template <int MODE> struct RingVmax<float, MODE> {
     static constexpr int one = kAcc ? 4 : 6, shared = kAcc ? 4 : 5;
 };
 
-// Row warps (rows per tile) and column warps of the split backward
-// (ln_split.cuh), and the widest row it serves in 16-byte vectors per lane of
-// a row warp.  It takes 16-bit rows of LN_SPLIT_FROM_V .. kSplitMaxV vectors
-// per lane in the plain and dinp-accumulating backward; with
-// recomputed statistics (the column warps would need the row warps' results
-// first) those rows stay on the shared-row ring.  8 + 4 warps and the
-// producer: ptxas fits the layout in 128 registers without spilling (13 warps
-// x 32 x 128 of the SM's 65536), and 8-row stages of bf16 C = 1600 leave room
-// for a 4-deep ring.
-// Measured on B200 (bf16, back-to-back calls): C = 2048 26.7 us against 28.3
-// on the shared-row ring, C = 1600 40.0 against 39.6 (accumulating 43.6
-// against 45.2), C = 1280 33.1 against 27.7, C = 1024 46.2 against 41.6 (one
-// warp per row); so rows from 7 vectors per lane.
+// The split backward (ln_split.cuh): 8 row warps (rows per tile), column
+// warps and the producer.  It takes 16-bit rows of LN_SPLIT_FROM_V ..
+// kSplitMaxV vectors per row-warp lane in the plain and dinp-accumulating
+// backward; with recomputed statistics (the column warps would need the row
+// warps' results first) those rows stay on the shared-row ring.  At most 16
+// warps, so that ptxas can give every thread 128 registers (one scheduler's
+// 16384 registers over 4 warps); the row warps keep g = dout * weight
+// unpacked (up to 64 of them).
+// Measured on B200 (bf16, back-to-back calls, median of 7 interleaved rounds,
+// against the ring kernel): C = 2048 25.5 us against 28.4, C = 1600 36.9
+// against 39.6; C = 1536 34.9 against 35.0, C = 1280 27.9 against 27.6,
+// C = 1152 31.8 against 30.9, C = 1024 44.9 against 41.9.  So rows from 7
+// vectors per lane.
 #ifndef LN_SPLIT_FROM_V
 #define LN_SPLIT_FROM_V 7
 #endif
 constexpr int kSplitRowWarps = 8;
-constexpr int kSplitColWarps = 4;
 constexpr int kSplitMaxV = 8;
 template <typename T, int MODE> struct SplitServes {
     static constexpr bool value = sizeof(T) == 2 && (MODE & kBwdRecompute) == 0;
 };
+// Column warps for rows of up to 32 * VR vectors: one column vector per lane
+// (VR warps) while the block stays within 16 warps, else 4 warps of two.
+template <int VR> struct SplitCols {
+    static constexpr int value = kSplitRowWarps + VR + 1 <= 16 ? VR : 4;
+};
 // Column-warp vectors per lane for rows of 32 * VR vectors.
 template <int VR> struct SplitVc {
     static constexpr int value =
-        ((32 * VR + kSplitColWarps - 1) / kSplitColWarps + 31) / 32;
+        ((32 * VR + SplitCols<VR>::value - 1) / SplitCols<VR>::value + 31) / 32;
 };
 
 // Calls visitor.template ring<V, W>() or visitor.template split<VR, VC>();

@@ -159,7 +159,7 @@ struct BwdChoice {
     template <int VR, int VC>
     void split() {
         const int C = nvec * E;
-        constexpr int NR = lnk::kSplitRowWarps, NCOL = lnk::kSplitColWarps;
+        constexpr int NR = lnk::kSplitRowWarps, NCOL = lnk::SplitCols<VR>::value;
         const int S = lnk::split_stages<T, NR, NS>(C, kMax);
         label = "split VR=" + num(VR) + " VC=" + num(VC) + " S=" + num(S);
         check(lnk::SplitServes<T, MODE>::value, ctx() + "split rows: 16-bit, statistics read");
@@ -171,7 +171,7 @@ struct BwdChoice {
         check(2 * lnk::kSplitMaxStages * 8 <= 128, ctx() + "split barriers fit in 128 bytes");
         check(lnk::split_smem<T, NR, NS>(C, S) <= kMax, ctx() + "split shared memory fits");
         check(lnk::split_ring_offset(C) % 128 == 0, ctx() + "split ring starts 128-aligned");
-        check(32 * (NR + NCOL + 1) <= 1024, ctx() + "split block size");
+        check(NR + NCOL + 1 <= 16, ctx() + "split block of at most 16 warps (128 registers)");
         check_copies(ctx(), size_t(C) * sizeof(T), NR, NS);
     }
     template <int V, int W, int G>

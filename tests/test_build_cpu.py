@@ -33,6 +33,12 @@ NO_SPILL = {
     "backward fp16 C=768": "_ZN3lnk17ln_bwd_tma_kernelI6__halfLi3ELi15ELi4ELb1ELi1ELi0E",
     "backward fp32 C=768 (ring, 6 vectors)":
         "_ZN3lnk17ln_bwd_tma_kernelIfLi6ELi15ELi2ELb1ELi1ELi0E",
+    "backward bf16 C=1600 (split: 8 row warps, 7 column warps)":
+        "_ZN3lnk19ln_bwd_split_kernelI13__nv_bfloat16Li7ELi1ELi8ELi7ELi0E",
+    "accumulating backward bf16 C=1600 (split)":
+        "_ZN3lnk19ln_bwd_split_kernelI13__nv_bfloat16Li7ELi1ELi8ELi7ELi1E",
+    "backward bf16 C=2048 (split: 8 row warps, 4 column warps)":
+        "_ZN3lnk19ln_bwd_split_kernelI13__nv_bfloat16Li8ELi2ELi8ELi4ELi0E",
     "column finalise": "_ZN3lnk16ln_colsum_kernelEPfS0_PKfiii",
 }
 # Every kernel: spill stores and loads, and the stack frame, at most this

@@ -81,8 +81,8 @@ PINNED = [
     ("fwd", "bf16", 0, 2000, "vec V=4 W=16"),            # C = 16000
     ("bwd", "bf16", 0, 96, "ring V=3 W=1 S=4"),          # GPT-2 124M
     ("bwd", "bf16", 0, 128, "ring V=4 W=1 S=3"),         # GPT-2 350M
-    ("bwd", "bf16", 0, 200, "split VR=7 VC=2 S=4"),      # GPT-2 1.5B: row and column warps
-    ("bwd", "bf16", 1, 200, "split VR=7 VC=2 S=2"),      # accumulating 1.5B: three arrays
+    ("bwd", "bf16", 0, 200, "split VR=7 VC=1 S=4"),      # GPT-2 1.5B: 8 row, 7 column warps
+    ("bwd", "bf16", 1, 200, "split VR=7 VC=1 S=2"),      # accumulating 1.5B: three arrays
     ("bwd", "bf16", 2, 200, "ring V=3 W=3 S=4"),         # recomputing 1.5B: three warps per row
     ("bwd", "f32", 0, 192, "ring V=6 W=1 S=2"),          # fp32, C = 768
     ("bwd", "bf16", 1, 96, "ring V=3 W=1 S=3"),          # accumulating: three arrays a stage
