@@ -48,7 +48,8 @@
  *     a multiple of 16 bytes take the vectorised path; others a scalar path.
  *   - Errors are returned as an ln_status value; nothing is launched when
  *     validation fails, and no kernel asserts or traps.
- *   - Calls can be captured into a CUDA graph (the backward's workspace then
+ *   - ln_forward, ln_forward_residual, ln_backward and ln_backward_ex calls
+ *     can be captured into a CUDA graph (the backward's workspace then
  *     becomes graph allocation nodes); make one uncaptured call of the same
  *     shape on the device first, so that one-time set-up (the device's memory
  *     pool, kernel attributes) happens outside the capture.
@@ -204,7 +205,8 @@ int ln_backward_ex(void *dinp, float *dweight, float *dbias, const void *dout,
  * stream-ordered pool; this variant keeps them in a static device array of
  * LN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
  * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
- * other allocating routine.
+ * other allocating routine, and does not create the memory pool that
+ * ln_backward uses (a process that only calls this entry point has none).
  *   - The first call on a device (made with that device current) looks up the
  *     array's device address once; make that call before any stream capture.
  *   - All calls share the one array.  Each call overwrites what it reads, so
