@@ -9,7 +9,7 @@
 // Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
 // persistent TMA-ring kernel (ln_tma.cuh) on one warp per row; 16-bit rows of
 // 7..8 vectors per lane (plain and accumulating) the split ring of row and
-// column warps (ln_split.cuh); other wider rows the ring with W = 2..4 warps
+// column warps (ln_split.cuh); other wider rows the ring with W = 2..7 warps
 // per row; rows wider than that take the register-resident kernel (W =
 // 4..16 warps per row, 4 vectors per thread).
 // Rows wider than the widest variant, and any misaligned call, take the
@@ -191,8 +191,17 @@ template <int VR> struct SplitVc {
         ((32 * VR + SplitCols<VR>::value - 1) / SplitCols<VR>::value + 31) / 32;
 };
 
+// Shared rows of the ring: up to kRingMaxW warps per row (15, 12 or 14
+// consumer warps at W = 5, 6, 7: whole row groups within the 16-warp block).
+// Past that the register-resident kernels take over.
+#ifndef LN_RING_MAX_W
+#define LN_RING_MAX_W 7
+#endif
+constexpr int kRingMaxW = LN_RING_MAX_W;
+static_assert(kRingMaxW == 4 || kRingMaxW == 7, "ring widths: up to 4 or 7 warps per row");
+
 // Calls visitor.template ring<V, W>() or visitor.template split<VR, VC>();
-// false when rows are wider than 4 warps of the ring cover.
+// false when rows are wider than kRingMaxW warps of the ring cover.
 template <typename T, int MODE, typename Visitor>
 bool visit_bwd_ring(int nvec, Visitor &v) {
     constexpr int NS = BwdRingArrays<MODE>::value;
@@ -202,6 +211,12 @@ bool visit_bwd_ring(int nvec, Visitor &v) {
     static_assert(bwd_ring_smem_max<T, VS, 2, NS>() <= kMaxSmemPerBlock, "ring fits");
     static_assert(bwd_ring_smem_max<T, VS, 3, NS>() <= kMaxSmemPerBlock, "ring fits");
     static_assert(bwd_ring_smem_max<T, VS, 4, NS>() <= kMaxSmemPerBlock, "ring fits");
+    static_assert(kRingMaxW < 5 || bwd_ring_smem_max<T, VS, 5, NS>() <= kMaxSmemPerBlock,
+                  "ring fits");
+    static_assert(kRingMaxW < 6 || bwd_ring_smem_max<T, VS, 6, NS>() <= kMaxSmemPerBlock,
+                  "ring fits");
+    static_assert(kRingMaxW < 7 || bwd_ring_smem_max<T, VS, 7, NS>() <= kMaxSmemPerBlock,
+                  "ring fits");
     const int v1 = (nvec + 31) / 32;
     if constexpr (SplitServes<T, MODE>::value) {
         if (v1 >= LN_SPLIT_FROM_V && v1 <= kSplitMaxV) {
@@ -233,11 +248,20 @@ bool visit_bwd_ring(int nvec, Visitor &v) {
         case 2: v.template ring<VS, 2>(); return true;
         case 3: v.template ring<VS, 3>(); return true;
         case 4: v.template ring<VS, 4>(); return true;
-        default: return false;
+        default: break;
     }
+    if constexpr (kRingMaxW >= 7) {
+        switch (w) {
+            case 5: v.template ring<VS, 5>(); return true;
+            case 6: v.template ring<VS, 6>(); return true;
+            case 7: v.template ring<VS, 7>(); return true;
+            default: break;
+        }
+    }
+    return false;
 }
 
-// Backward rows wider than the ring covers (more than 4 * 32 * shared
+// Backward rows wider than the ring covers (more than kRingMaxW * 32 * shared
 // vectors): the register-resident kernel with W = 4, 8 or 16 warps per row
 // and 4 vectors per thread.  Calls visitor.template run<V, W, GROUPS>();
 // false when rows are wider still.

@@ -178,7 +178,7 @@ struct BwdChoice {
     void run() {
         const int C = nvec * E;
         label = "vec V=" + num(V) + " W=" + num(W);
-        check(nvec > 4 * 32 * VS && nvec > 32 * ONE,
+        check(nvec > lnk::kRingMaxW * 32 * VS && nvec > 32 * ONE,
               ctx() + "the register-resident backward serves only rows past the ring");
         check(32 * W * V >= nvec, ctx() + "register-resident rows are covered");
         check(W == 4 || 32 * (W / 2) * V < nvec,

@@ -89,7 +89,9 @@ PINNED = [
     ("bwd", "bf16", 2, 96, "ring V=3 W=1 S=4"),          # recomputing
     ("bwd", "bf16", 2, 128, "ring V=3 W=2 S=4"),         # recomputing C = 1024: two warps
     ("bwd", "f16", 0, 96, "ring V=3 W=1 S=4"),           # fp16 GPT-2 124M shape
-    ("bwd", "bf16", 0, 512, "vec V=4 W=4"),              # C = 4096: past the ring
+    ("bwd", "bf16", 0, 512, "ring V=3 W=6 S=5"),         # C = 4096: six warps per row
+    ("bwd", "bf16", 0, 672, "ring V=3 W=7 S=4"),         # C = 5376: the ring's widest row
+    ("bwd", "bf16", 0, 673, "vec V=4 W=8"),              # past the ring
 ]
 
 
