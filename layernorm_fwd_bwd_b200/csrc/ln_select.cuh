@@ -127,7 +127,7 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
 }
 
 // Backward ring (ln_tma.cuh).  One warp per row while a lane holds at most
-// `one` vectors; wider rows are split over W = 2..4 warps with `shared`
+// `one` vectors; wider rows are split over W = 2..7 warps with `shared`
 // vectors per lane, which keeps x - mean in registers between the two
 // passes.  Measured on B200: bf16 C = 1024 is faster on one warp (4 vectors,
 // recomputing x - mean) than on two (the row-group exchange costs more than
