@@ -98,19 +98,41 @@ struct FwdVec {
             run<4, 4, 2>();
         }
     }
+    // Rows of 17..32 vectors per lane on four warps per row (V per warp):
+    // blocks of 16 warps (4 rows per tile, 128 registers per thread) with as
+    // many tiles (1..3) as fit in shared memory.  Measured on B200 (bf16,
+    // 500 back-to-back calls) against the register-resident kernel with 8
+    // warps per row: C = 8192 30.0 us against 38.3 (N = 4096), 98.2 against
+    // 123.0 (N = 16384); C = 6144 32.4 against 37.7; C = 5120 35.1 against
+    // 37.3; C = 4608 39.6 against 38.4.  Preferring fewer tiles so that two
+    // blocks share an SM was slower at every width (34-51 us).
+    template <int V>
+    void run_tile_four() {
+        constexpr int RW = 4, NW = 16;
+        if (ceil_div(a.N, NW / RW) > INT32_MAX) {
+            run<4, 8, 1>();
+        } else if (lnk::fwd_tile_smem<T, NW, 3, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+            run_tile<V, RW, 3, NW>();
+        } else if (lnk::fwd_tile_smem<T, NW, 2, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+            run_tile<V, RW, 2, NW>();
+        } else if (lnk::fwd_tile_smem<T, NW, 1, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+            run_tile<V, RW, 1, NW>();
+        } else {
+            run<4, 8, 1>();
+        }
+    }
     // Rows that fill every lane's V vectors exactly take a variant without
     // per-vector bound checks.
-    template <int V, int RW, int TL = lnk::kTileFwdTiles>
+    template <int V, int RW, int TL = lnk::kTileFwdTiles, int NWB = lnk::kTileWarps * RW>
     void run_tile() {
         constexpr int E = lnk::Vec<T>::E;
         if (a.C / E == 32 * RW * V)
-            run_tile_k<V, RW, TL, true>();
+            run_tile_k<V, RW, TL, true, NWB>();
         else
-            run_tile_k<V, RW, TL, false>();
+            run_tile_k<V, RW, TL, false, NWB>();
     }
-    template <int V, int RW, int TL, bool FULL>
-    void run_tile_k() {
-        constexpr int NW = lnk::kTileWarps * RW;          // 8 rows per tile either way
+    template <int V, int RW, int TL, bool FULL, int NW = lnk::kTileWarps * RW>
+    void run_tile_k() {   // NW warps: NW / RW rows per tile (8 for one or two warps per row)
         auto kern = lnk::ln_fwd_tile_kernel<T, V, NW, TL, RW, FULL, MODE>;
         const int threads = 32 * NW;
         const size_t smem = lnk::fwd_tile_smem<T, NW, TL, RW, kArrays>(a.C);

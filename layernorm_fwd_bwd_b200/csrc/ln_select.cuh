@@ -4,8 +4,8 @@
 //
 // Forward: rows of up to 8 vectors per lane take the one-shot tile kernel
 // (ln_tile.cuh) with one warp per row, rows of 9..16 the same kernel with two
-// warps per row; wider rows take the persistent register-resident kernel
-// with W = 4, 8 or 16 warps per row and 4 vectors per thread.
+// warps per row, rows of 17..32 with four; wider rows take the persistent
+// register-resident kernel with 16 warps per row and 4 vectors per thread.
 // Backward: rows of up to 4 (bf16, fp16) / 6 (fp32) vectors per lane take the
 // persistent TMA-ring kernel (ln_tma.cuh) on one warp per row; 16-bit rows of
 // 7..8 vectors per lane (plain and accumulating) the split ring of row and
@@ -62,6 +62,11 @@ template <int W> struct BwdRingConsumers {
 #ifndef LN_TILE_FWD_TWO_WARPS
 #define LN_TILE_FWD_TWO_WARPS 1
 #endif
+// Rows of 17..32 vectors per lane (bf16 C = 4097..8192): the tile kernel with
+// four warps per row instead of the register-resident kernel with eight.
+#ifndef LN_TILE_FWD_FOUR_WARPS
+#define LN_TILE_FWD_FOUR_WARPS 1
+#endif
 constexpr int kTileWarps = 8;   // rows per forward tile (warps per tile, doubled at two per row)
 constexpr int kTileFwdTiles = LN_TILE_FWD_TILES;
 
@@ -117,6 +122,15 @@ bool visit_fwd_vec(int nvec, Visitor &v) {
             case 6: v.template run_tile_two<6>(); return true;
             case 7: v.template run_tile_two<7>(); return true;
             case 8: v.template run_tile_two<8>(); return true;
+            default: break;
+        }
+    }
+    if constexpr (LN_TILE_FWD_FOUR_WARPS) {
+        switch ((nvec + 127) / 128) {        // vectors per lane on four warps per row
+            case 5: v.template run_tile_four<5>(); return true;
+            case 6: v.template run_tile_four<6>(); return true;
+            case 7: v.template run_tile_four<7>(); return true;
+            case 8: v.template run_tile_four<8>(); return true;
             default: break;
         }
     }

@@ -97,6 +97,8 @@ struct FwdChoice {
                   ctx() + "register-resident rows take the fewest warps");
             check(!LN_TILE_FWD_TWO_WARPS || nvec > 2 * 32 * 8,
                   ctx() + "rows of up to 16 vectors per lane take the two-warp tile");
+            check(!LN_TILE_FWD_FOUR_WARPS || nvec > 4 * 32 * 8,
+                  ctx() + "rows of up to 32 vectors per lane take the four-warp tile");
             check(lnk::fwd_vec_smem<W, G>(C) <= kMax, ctx() + "register-resident smem fits");
         }
     }
@@ -116,6 +118,24 @@ struct FwdChoice {
         check_copies(ctx() + "weight and bias: ", size_t(C) * sizeof(T), 1, 2);
         check(nvec <= 4 * 32 * 4 && lnk::fwd_vec_smem<4, 2>(C) <= kMax,
               ctx() + "the four-warp register-resident fallback covers the row");
+    }
+    template <int V>
+    void run_tile_four() {
+        const int C = nvec * E;
+        constexpr int NW = 16, RW = 4;
+        int tl = 0;
+        if (lnk::fwd_tile_smem<T, NW, 3, RW, kArrays>(C) <= kMax) tl = 3;
+        else if (lnk::fwd_tile_smem<T, NW, 2, RW, kArrays>(C) <= kMax) tl = 2;
+        else if (lnk::fwd_tile_smem<T, NW, 1, RW, kArrays>(C) <= kMax) tl = 1;
+        label = "tile4 V=" + num(V) + " W=4 tiles=" + num(tl);
+        check(128 * V >= nvec && 128 * (V - 1) < nvec,
+              ctx() + "four-warp rows take the fewest vectors per lane");
+        check(nvec > 2 * 32 * 8, ctx() + "four-warp rows are wider than two warps serve");
+        check(tl >= 1, ctx() + "a one-tile four-warp block fits");
+        check_copies(ctx(), size_t(C) * sizeof(T), NW / RW, kArrays);
+        check_copies(ctx() + "weight and bias: ", size_t(C) * sizeof(T), 1, 2);
+        check(nvec <= 8 * 32 * 4 && lnk::fwd_vec_smem<8, 1>(C) <= kMax,
+              ctx() + "the eight-warp register-resident fallback covers the row");
     }
 };
 

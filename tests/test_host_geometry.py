@@ -78,6 +78,9 @@ PINNED = [
     ("fwd", "bf16", 0, 384, "tile2 V=6 W=2"),            # C = 3072: two warps per row
     ("fwd", "bf16", 0, 512, "tile2 V=8 W=2"),            # C = 4096
     ("fwd", "bf16", 1, 512, "tile2 V=8 W=2 tiles=1"),    # residual C = 4096: one tile
+    ("fwd", "bf16", 0, 1024, "tile4 V=8 W=4 tiles=3"),   # C = 8192: four warps per row
+    ("fwd", "bf16", 1, 1024, "tile4 V=8 W=4 tiles=1"),   # residual C = 8192: two arrays
+    ("fwd", "bf16", 0, 1025, "vec V=4 W=16"),            # past the four-warp tile
     ("fwd", "bf16", 0, 2000, "vec V=4 W=16"),            # C = 16000
     ("bwd", "bf16", 0, 96, "ring V=3 W=1 S=4"),          # GPT-2 124M
     ("bwd", "bf16", 0, 128, "ring V=4 W=1 S=3"),         # GPT-2 350M

@@ -129,6 +129,20 @@ def test_split_backward_widths(lib, dtype, C, N):
     _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
 
 
+# Forward rows of 17..32 vectors per lane on four warps per row (16-bit C =
+# 4104..8192, fp32 C = 2052..4096), one to three tiles per block; N = 5 is one
+# partial tile, N = 1003 several blocks with a ragged last one.
+FOUR_C = {"bf16": [4104, 5008, 6144, 8192], "f16": [4104, 8192], "f32": [2056, 3000, 4096]}
+
+
+@pytest.mark.parametrize("dtype,C", [(d, c) for d, cs in FOUR_C.items() for c in cs])
+@pytest.mark.parametrize("N", [5, 1003])
+def test_four_warp_forward_widths(lib, dtype, C, N):
+    batch = wl.custom(dtype, N, C, seed=7000 + C + N)
+    dev, _, ref_stats, _ = _forward_parity(lib, batch, f"{dtype} {N}x{C}", scaled=True)
+    _backward_parity(lib, batch, dev, f"{dtype} {N}x{C}", ref_stats, scaled=True)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_widest_row(lib, dtype):
     """C = LN_MAX_C (2^24 channels, 32 or 64 MB a row), two rows, every

@@ -124,7 +124,7 @@ def test_backward_variants_full(lib, name, flags):
     print(_backward_ex(lib, batch, extras, FLAG_SETS[flags], f"{name} {flags}"))
 
 
-SWEEP_C = [1, 3, 8, 33, 128, 512, 768, 1024, 1600, 2056, 3072, 4096, 20000]
+SWEEP_C = [1, 3, 8, 33, 128, 512, 768, 1024, 1600, 2056, 3072, 4096, 6144, 8192, 20000]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
