@@ -17,8 +17,8 @@
 // are separated, and both read the same shared-memory stages:
 //   * NR row warps, one row each per tile (tile = NR consecutive rows): the
 //     row sums S1 = sum g, S2 = sum g * (x - mean) (g = dout * weight) and
-//     dinp.  They hold the packed row in registers from the stage read to
-//     the dinp store, and no accumulator at all.
+//     dinp.  They keep g unpacked in registers between the two passes, read
+//     x again from the stage in pass 2, and hold no accumulator at all.
 //   * NCOL column warps, each owning a fixed slice of about nvec / NCOL
 //     16-byte column vectors for the whole launch: for every row of every
 //     tile, in row order, they add dout * xhat and dout into their slice's
@@ -30,11 +30,12 @@
 //     previous dinp when accumulating) with 1-D bulk copies (cp.async.bulk,
 //     no multicast) into S stages; S is as many as fit in the block's shared
 //     memory (read back from %dynamic_smem_size, 2..8).
-// A stage is free once every row warp has read its row (after pass 2 when
-// the stage also holds the previous dinp) and every column warp has passed
-// over all its rows: its "empty" mbarrier counts NR + NCOL arrivals, each
-// after a fence.proxy.async that orders the warp's reads before the next
-// bulk copy into the stage.  Waits are bounded exactly as in ln_tma.cuh.
+// A stage is free once every row warp has finished its row (pass 2 reads x,
+// and the previous dinp when accumulating, from the stage) and every column
+// warp has passed over all its rows: its "empty" mbarrier counts NR + NCOL
+// arrivals, each after a fence.proxy.async that orders the warp's reads
+// before the next bulk copy into the stage.  Waits are bounded exactly as in
+// ln_tma.cuh.
 #pragma once
 
 #include "ln_tma.cuh"
