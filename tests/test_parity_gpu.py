@@ -161,8 +161,10 @@ def test_widest_row(lib, dtype):
 BEYOND_INT32 = [("bf16", 768, 4096, 700),    # tile forward, ring backward
                 ("f32", 768, 4096, 700),     # the same kernels, 8.8 GB arrays
                 ("bf16", 770, 4096, 700),    # scalar kernels (C * 2 not a multiple of 16)
-                ("bf16", 4096, 1024, 520),   # two-warp tile forward, register-resident backward
-                ("bf16", 16000, 256, 560)]   # register-resident kernels, 16 warps per row
+                ("bf16", 4096, 1024, 520),   # two-warp tile forward, six-warp ring backward
+                ("bf16", 16000, 256, 560),   # register-resident kernels, 16 warps per row
+                ("bf16", 1600, 4096, 330),   # split backward (row and column warps)
+                ("bf16", 8192, 256, 1030)]   # four-warp tile forward, register-resident backward
 
 
 @pytest.mark.parametrize("dtype,C,P,k", BEYOND_INT32)
