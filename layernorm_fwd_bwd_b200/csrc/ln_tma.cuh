@@ -196,8 +196,8 @@ __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, f
 // tile and, within it, vectors j = (w % W) * 32 + lane + i * 32 * W; it keeps
 // dout*xhat and dout for those columns in registers.  Row sums of the W warps
 // of a row meet in shared memory (group_exchange).  At the end the RT row
-// groups are added in a fixed tree (warps owning the same columns only) and
-// the warps of group 0 write the block's partial row.  mean/rstd of the next
+// groups park their column sums in shared memory and the whole block adds
+// them in group order and writes the block's partial row.  mean/rstd of the next
 // row are prefetched one tile ahead; with MODE & kBwdRecompute they are not
 // read at all but recomputed from the staged row (pivot x[r, 0], two-pass
 // deviations, as in the forward).
