@@ -443,6 +443,34 @@ def call_loop_us(torch, stream, call, calls: int = LOOP_CALLS) -> float:
     return start.elapsed_time(end) * 1e3 / calls
 
 
+def graph_loop_us(torch, stream, call, calls: int = 200, reps: int = 3) -> float:
+    """Mean duration of one call when `calls` back-to-back calls are captured
+    in one CUDA graph on `stream` and the graph is replayed there (median of
+    `reps` replays, each timed with CUDA events on that stream, after one
+    untimed replay)."""
+    for i in range(4):
+        call(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(calls):
+            call(i)
+    times = []
+    with torch.cuda.stream(stream):
+        g.replay()
+        torch.cuda.synchronize()
+        for _ in range(reps):
+            start = torch.cuda.Event(enable_timing=True)
+            end = torch.cuda.Event(enable_timing=True)
+            start.record(stream)
+            g.replay()
+            end.record(stream)
+            torch.cuda.synchronize()
+            times.append(start.elapsed_time(end) * 1e3 / calls)
+    del g
+    return sorted(times)[len(times) // 2]
+
+
 def variant_bytes(w) -> dict:
     """Compulsory HBM bytes of one call of each variant (s = element size):
     residual forward reads resid and branch and writes resid_out and out
@@ -530,12 +558,18 @@ def run_variants(torch, ln, stream, sets, weight, bias, dweight, dbias, w, eps, 
 
 
 def run_workloads(torch, ln, stream, dev, nsets: int, calls: int = LOOP_CALLS) -> dict:
-    """ln_forward and ln_backward on every workload at its full size, each
-    timed like the headline's fwd and bwd: `calls` back-to-back calls over
-    rotating buffer sets (a backward reads a set whose forward ran
-    ``nsets // 2`` calls earlier), CUDA events around the loop on the
-    launching stream.  GB/s counts compulsory bytes; ``frac`` is against the
-    measured HBM copy bandwidth (or the fallback, as ``peak_kind`` says)."""
+    """ln_forward and ln_backward on every workload at its full size, timed
+    like the headline: `calls` back-to-back calls over rotating buffer sets
+    (a backward reads a set whose forward ran ``nsets // 2`` calls earlier),
+    CUDA events around the loop on the launching stream.  ``fwd_us`` and
+    ``bwd_us`` time loops of one call kind; ``step_us`` times the step itself,
+    forward and backward alternating as in the headline's timed region, and
+    ``GB_s``, ``frac`` and ``rows_per_s`` come from it.  ``graph_step_us`` is
+    the same step loop captured in one CUDA graph and replayed (the library's
+    calls are capturable), which removes the host's launch path but not the
+    kernels' own boundaries.  GB/s counts compulsory bytes; ``frac`` is
+    against the measured HBM copy bandwidth (or the fallback, as
+    ``peak_kind`` says)."""
     import numpy as np
 
     from layernorm_fwd_bwd_b200 import workloads as wl
@@ -585,20 +619,29 @@ def run_workloads(torch, ln, stream, dev, nsets: int, calls: int = LOOP_CALLS) -
             if rc:
                 raise ln.LNError(rc)
 
+        def step(i):
+            fwd(i)
+            bwd(i)
+
         for k in range(nsets):
             fwd(k)
         f_us = call_loop_us(torch, stream, fwd, calls)
         b_us = call_loop_us(torch, stream, bwd, calls)
+        s_us = call_loop_us(torch, stream, step, calls)
+        g_us = graph_loop_us(torch, stream, step)
         fb, bb = w.fwd_bytes(), w.bwd_bytes()
-        step_gbs = (fb + bb) / ((f_us + b_us) * 1e-6) / 1e9
+        step_gbs = (fb + bb) / (s_us * 1e-6) / 1e9
+        graph_gbs = (fb + bb) / (g_us * 1e-6) / 1e9
         out[name] = {
             "N": N, "C": C, "dtype": w.dtype,
             "fwd_us": round(f_us, 3), "bwd_us": round(b_us, 3),
+            "step_us": round(s_us, 3), "graph_step_us": round(g_us, 3),
             "fwd_GB_s": round(fb / (f_us * 1e-6) / 1e9, 1),
             "bwd_GB_s": round(bb / (b_us * 1e-6) / 1e9, 1),
-            "GB_s": round(step_gbs, 1), "rows_per_s": round(N / ((f_us + b_us) * 1e-6), 1),
+            "GB_s": round(step_gbs, 1), "rows_per_s": round(N / (s_us * 1e-6), 1),
             "frac": round(step_gbs / peak, 4),
             "bwd_frac": round(bb / (b_us * 1e-6) / 1e9 / peak, 4),
+            "graph_GB_s": round(graph_gbs, 1), "graph_frac": round(graph_gbs / peak, 4),
             "bytes": fb + bb,
             "l2": ("inputs smaller than L2: launch-bound correctness case"
                    if nsets * 2 * N * C * w.elem_bytes < 126e6 else
