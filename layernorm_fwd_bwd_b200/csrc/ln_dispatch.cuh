@@ -50,6 +50,12 @@ inline int tile_rows_per_block(int64_t N, int max_rows, int64_t resident) {
     return best;
 }
 
+// Whether every block count that tile_rows_per_block can pick for `max_rows`
+// (at least half of it per block) fits the grid's x dimension.
+inline bool tile_grid_fits(int64_t N, int max_rows) {
+    return ceil_div(N, (max_rows + 1) / 2) <= INT32_MAX;
+}
+
 template <typename T, int MODE>
 struct FwdVec {
     const FwdArgs &a;
@@ -59,11 +65,11 @@ struct FwdVec {
     template <int V, int W, int GROUPS>
     void run() {
         if constexpr (W == 1) {
-            if (ceil_div(a.N, lnk::kTileWarps) <= INT32_MAX) {
-                if constexpr (V >= LN_TILE_FWD_W2_FROM_V)
-                    run_tile<(V + 1) / 2, 2>();
-                else
-                    run_tile<V, 1>();
+            if constexpr (V >= LN_TILE_FWD_W2_FROM_V) {
+                run_tile_two<(V + 1) / 2>();
+                return;
+            } else if (tile_grid_fits(a.N, lnk::kTileWarps * lnk::kTileFwdTiles)) {
+                run_tile<V, 1>();
                 return;
             }
         }
@@ -88,11 +94,12 @@ struct FwdVec {
     void run_tile_two() {
         constexpr int NW = lnk::kTileWarps * 2;
         constexpr int TL = lnk::kTileFwdTiles;
-        if (ceil_div(a.N, lnk::kTileWarps) > INT32_MAX) {
-            run<4, 4, 2>();
-        } else if (lnk::fwd_tile_smem<T, NW, TL, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+        constexpr int RT = NW / 2;   // rows per tile
+        if (lnk::fwd_tile_smem<T, NW, TL, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock &&
+            tile_grid_fits(a.N, RT * TL)) {
             run_tile<V, 2>();
-        } else if (lnk::fwd_tile_smem<T, NW, 1, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+        } else if (lnk::fwd_tile_smem<T, NW, 1, 2, kArrays>(a.C) <= lnk::kMaxSmemPerBlock &&
+                   tile_grid_fits(a.N, RT)) {
             run_tile<V, 2, 1>();
         } else {
             run<4, 4, 2>();
@@ -108,14 +115,15 @@ struct FwdVec {
     // blocks share an SM was slower at every width (34-51 us).
     template <int V>
     void run_tile_four() {
-        constexpr int RW = 4, NW = 16;
-        if (ceil_div(a.N, NW / RW) > INT32_MAX) {
-            run<4, 8, 1>();
-        } else if (lnk::fwd_tile_smem<T, NW, 3, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+        constexpr int RW = 4, NW = 16, RT = NW / RW;   // RT rows per tile
+        if (lnk::fwd_tile_smem<T, NW, 3, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock &&
+            tile_grid_fits(a.N, RT * 3)) {
             run_tile<V, RW, 3, NW>();
-        } else if (lnk::fwd_tile_smem<T, NW, 2, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+        } else if (lnk::fwd_tile_smem<T, NW, 2, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock &&
+                   tile_grid_fits(a.N, RT * 2)) {
             run_tile<V, RW, 2, NW>();
-        } else if (lnk::fwd_tile_smem<T, NW, 1, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock) {
+        } else if (lnk::fwd_tile_smem<T, NW, 1, RW, kArrays>(a.C) <= lnk::kMaxSmemPerBlock &&
+                   tile_grid_fits(a.N, RT)) {
             run_tile<V, RW, 1, NW>();
         } else {
             run<4, 8, 1>();

@@ -280,6 +280,27 @@ void rows_per_block_all() {
             }
     check(lnh::tile_rows_per_block(16384, 16, 444) == 13,
           "GPT-2 1.5B forward: 13 rows per block on 444 resident blocks");
+
+    // tile_grid_fits accepts a row count exactly when every rows-per-block
+    // choice gives a block count that fits the grid's x dimension.
+    const int64_t I = INT32_MAX;
+    for (int max_rows : {4, 8, 12, 16})
+        for (int64_t k = 1; k <= 16; ++k)
+            for (int64_t d = -3; d <= 3; ++d) {
+                const int64_t N = k * I + d;
+                if (N < 1) continue;
+                bool all_fit = true;
+                for (int rows = (max_rows + 1) / 2; rows <= max_rows; ++rows)
+                    all_fit = all_fit && (N + rows - 1) / rows <= I;
+                check(lnh::tile_grid_fits(N, max_rows) == all_fit,
+                      "tile_grid_fits(" + num(N) + ", " + num(max_rows) + ")");
+                if (lnh::tile_grid_fits(N, max_rows))
+                    for (int64_t res : residents) {
+                        const int rows = lnh::tile_rows_per_block(N, max_rows, res);
+                        check((N + rows - 1) / rows <= I, "tile grid of " + num(N) +
+                                                              " rows fits the x dimension");
+                    }
+            }
 }
 
 }  // namespace
