@@ -85,6 +85,15 @@ __device__ __forceinline__ void warp_sum2(float &a, float &b) {
     }
 }
 
+__device__ __forceinline__ void warp_sum3(float &a, float &b, float &c) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+    }
+}
+
 // Block-wide sums for the scalar kernels (blockDim.x a multiple of 32).
 __device__ __forceinline__ float block_sum(float v, float *slot, int nwarps) {
     v = warp_sum(v);

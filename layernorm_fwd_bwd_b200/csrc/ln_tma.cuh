@@ -129,7 +129,7 @@ __host__ __device__ constexpr size_t bwd_tma_smem(int C) {
     // issue slots than the wider shared-memory reads), the ring, and the
     // row-group exchange slots when rows are shared by W > 1 warps
     return tma_ring_offset<T>(C) + align128(bwd_tma_ring_bytes<T, NC, S, W, NS>(C)) +
-           (W > 1 ? size_t(NC / W) * 2 * 3 * W * 4 : 0);
+           (W > 1 ? size_t(NC / W) * 2 * 4 * W * 4 : 0);
 }
 
 // Producer side: stream tiles k = 0, 1, ... of this
@@ -160,7 +160,8 @@ __device__ __forceinline__ void tma_produce(uint64_t *full, uint64_t *empty,
 // sums (a, b) and an abort flag into a slot of its group, the group meets at a
 // named barrier, and every warp reads all W entries in the same order.  Slots
 // alternate by parity, so a slot is rewritten only after every warp of the
-// group has passed the next barrier (and so has read it).
+// group has passed the next barrier (and so has read it).  A slot holds 3W
+// floats here and 4W in group_exchange3 (three sums and the flag).
 template <int W>
 __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, float *slot,
                                                int group, int sub, int lane) {
@@ -186,6 +187,34 @@ __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, f
     }
 }
 
+template <int W>
+__device__ __forceinline__ bool group_exchange3(float &a, float &b, float &c, bool abort,
+                                                float *slot, int group, int sub, int lane) {
+    if constexpr (W == 1) {
+        return abort;
+    } else {
+        if (lane == 0) {
+            slot[4 * sub + 0] = a;
+            slot[4 * sub + 1] = b;
+            slot[4 * sub + 2] = c;
+            slot[4 * sub + 3] = abort ? 1.f : 0.f;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(group + 1), "r"(32 * W) : "memory");
+        a = 0.f;
+        b = 0.f;
+        c = 0.f;
+        float any = 0.f;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            a += slot[4 * k + 0];
+            b += slot[4 * k + 1];
+            c += slot[4 * k + 2];
+            any += slot[4 * k + 3];
+        }
+        return any != 0.f;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Backward.  NC consumer warps (15 by default: with the producer warp a
 // 512-thread block, one per SM, 128 registers per thread), W warps per row,
@@ -206,6 +235,17 @@ __device__ __forceinline__ bool group_exchange(float &a, float &b, bool abort, f
 #ifndef LN_RING_KEEP_G_SHARED_PLAIN
 #define LN_RING_KEEP_G_SHARED_PLAIN 1
 #endif
+// Whether the recomputing backward, where it does not keep g, reduces the
+// row's variance together with its two backward sums (one butterfly and one
+// row exchange of three values instead of two in a row).  The variance's
+// per-lane sums and reduction order are the same, so mean and rstd are
+// bit-identical either way; dinp and dweight then take the form that scales
+// x - mean by rstd once per element (rounding differs in the last bits).
+// Where g is kept, the column sums would have to wait for pass 2 and the
+// packed dout would hold its registers until then: slower on B200.
+#ifndef LN_RING_FUSE_RECOMP_VAR
+#define LN_RING_FUSE_RECOMP_VAR 1
+#endif
 
 template <typename T, int V, int NC, int S, bool RR, int W = 1, int MODE = 0>
 __global__ void __launch_bounds__(32 * (NC + 1), (NC + 1) * 32 <= 256 ? 2 : 1)
@@ -219,6 +259,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     static_assert(NC % W == 0 && NC / W >= 2 && NC / W <= 15, "row groups");
     constexpr bool ACC = (MODE & kBwdAccumulate) != 0;
     constexpr bool RECOMP = (MODE & kBwdRecompute) != 0;
+    // floats per warp in a row-exchange slot: 4 for group_exchange3
+    constexpr int XW = RECOMP ? 4 : 3;
     constexpr int NS = ACC ? 3 : 2;                          // arrays per stage
     constexpr int E = Vec<T>::E;
     constexpr int P = E / 2;
@@ -234,7 +276,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
     const uint32_t half_bytes = RT * row_bytes;              // one array of a stage
     const uint32_t stage_bytes = NS * half_bytes;
     float *s_red = reinterpret_cast<float *>(
-        ring + align128(bwd_tma_ring_bytes<T, NC, S, W, NS>(C)));   // [RT][2][3W] (W > 1)
+        ring + align128(bwd_tma_ring_bytes<T, NC, S, W, NS>(C)));   // [RT][2][4W] (W > 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int group = warp / W;                              // row in the tile
@@ -363,6 +405,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
             constexpr bool KEEP_G =
                 KEEP_D && (W == 1 || LN_RING_KEEP_G_SHARED_PLAIN) &&
                 (W == 1 || MODE == 0) && V <= (sizeof(T) == 4 ? (ACC ? 4 : 5) : (ACC ? 2 : 3));
+            constexpr bool FUSE_VAR = RECOMP && !KEEP_G && LN_RING_FUSE_RECOMP_VAR;
             uint4 *gr = reinterpret_cast<uint4 *>(dinp) + r * nvec;
             f32x2 d[KEEP_D ? V : 1][P];
             f32x2 gk[KEEP_G ? V : 1][P];
@@ -383,11 +426,14 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                     }
                 }
                 float a = warp_sum(hsum(sd)), unused = 0.f;
-                abort = group_exchange<W>(a, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                abort = group_exchange<W>(a, unused, abort, s_red + (group * 2 + parity) * XW * W,
                                           group, sub, lane);
                 parity ^= 1;
                 const float md = a * inv_C;
                 MD = pair(md, md);
+            }
+            if constexpr (RECOMP && !FUSE_VAR) {
+                float unused = 0.f;
                 f32x2 sq = pair(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
@@ -407,18 +453,25 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                     }
                 }
                 float v = warp_sum(hsum(sq));
-                abort = group_exchange<W>(v, unused, abort, s_red + (group * 2 + parity) * 3 * W,
+                abort = group_exchange<W>(v, unused, abort, s_red + (group * 2 + parity) * XW * W,
                                           group, sub, lane);
                 parity ^= 1;
                 s = rsqrtf(v * inv_C + eps);
             }
-            float *slot = s_red + (group * 2 + parity) * 3 * W;
+            float *slot = s_red + (group * 2 + parity) * XW * W;
             parity ^= 1;
-            const f32x2 Sx = pair(s, s);
-            f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f);
+            f32x2 Sx = pair(s, s);
+            f32x2 s1 = pair(0.f, 0.f), s2 = pair(0.f, 0.f), sq = pair(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int j = t + TPR * i;
+                if constexpr (FUSE_VAR && KEEP_D) {
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        d[i][q] = sub2(d[i][q], MD);
+                        if (j < nvec) sq = fma2(d[i][q], d[i][q], sq);
+                    }
+                }
                 if constexpr (KEEP_D && !RECOMP) {
                     // d for every slot (dead lanes' values are never used)
                     f32x2 dq[P];
@@ -454,19 +507,35 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                         for (int q = 0; q < P; ++q) {
                             f32x2 dq = sub2(x[q], K);
                             if constexpr (RECOMP) dq = sub2(dq, MD);
-                            const f32x2 xh = mul2(dq, Sx);
                             const f32x2 g = mul2(dy[q], wp[q]);
                             s1 = add2(s1, g);
-                            s2 = fma2(g, xh, s2);                 // sum g * xhat
+                            if constexpr (FUSE_VAR) {
+                                sq = fma2(dq, dq, sq);
+                                s2 = fma2(g, dq, s2);             // sum g * d
+                            } else {
+                                const f32x2 xh = mul2(dq, Sx);
+                                s2 = fma2(g, xh, s2);             // sum g * xhat
+                            }
                         }
                     }
                 }
             }
             float a = hsum(s1), b = hsum(s2);
-            warp_sum2(a, b);
-            abort = group_exchange<W>(a, b, abort, slot, group, sub, lane);
+            if constexpr (FUSE_VAR) {
+                float v = hsum(sq);
+                warp_sum3(a, b, v);
+                abort = group_exchange3<W>(a, b, v, abort, slot, group, sub, lane);
+                s = rsqrtf(v * inv_C + eps);
+                Sx = pair(s, s);
+            } else {
+                warp_sum2(a, b);
+                abort = group_exchange<W>(a, b, abort, slot, group, sub, lane);
+            }
             const float na = -s * (a * inv_C);
-            const float nc = KEEP_D ? -(s * s) * (s * (b * inv_C)) : -s * (b * inv_C);
+            // b is the sum of g * d (d = x - mean), or of g * xhat when
+            // pass 1 already knew rstd and did not keep d
+            constexpr bool B_OF_D = KEEP_D || FUSE_VAR;
+            const float nc = B_OF_D ? -(s * s) * (s * (b * inv_C)) : -s * (b * inv_C);
             const f32x2 NA = pair(na, na);
             const f32x2 NCc = pair(nc, nc);
 #pragma unroll
@@ -493,7 +562,10 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                                 f32x2 dq = sub2(pair_at<T>(xv[i], q), K);
                                 if constexpr (RECOMP) dq = sub2(dq, MD);
                                 xh = mul2(dq, Sx);
-                                o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
+                                if constexpr (FUSE_VAR)
+                                    o[q] = fma2(g, Sx, fma2(dq, NCc, NA));
+                                else
+                                    o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
                             }
                             acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
                             acc_b[i][q] = add2(acc_b[i][q], dy);
