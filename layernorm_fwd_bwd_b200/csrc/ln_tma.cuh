@@ -387,12 +387,15 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 continue;
             }
 
-            // Pass 1 / pass 2.  Where the register budget allows (KEEP_D), pass 1
-            // keeps d = x - mean as fp32 pairs and pass 2 evaluates
+            // Pass 1 / pass 2.  Pass 1 sums g = dout * weight and g * d over the
+            // row (d = x - mean) and pass 2 evaluates
             //   dinp = g*rstd + NA + d*NC,  NA = -rstd*mean(g),
-            //   NC = -rstd^3*mean(g*d)   (xhat = d*rstd),
-            // so pass 2 never unpacks x again; otherwise both passes rebuild
-            // xhat from the packed row.  Where it also allows (KEEP_G: one warp
+            //   NC = -rstd^3*mean(g*d)   (xhat = d*rstd).
+            // Where the register budget allows (KEEP_D), pass 1 keeps d as fp32
+            // pairs, so pass 2 never unpacks x again; otherwise both passes
+            // rebuild d from the packed row (summing g * d rather than g * xhat
+            // saves pass 1 a multiply per element: 41.0 -> 40.7 us at bf16
+            // C = 1024 on B200).  Where it also allows (KEEP_G: one warp
             // per row, or a shared row of the plain backward; narrow enough
             // rows), pass 1 keeps g = dout * weight too
             // and adds the row's dout * xhat and dout to the column sums, so
@@ -509,13 +512,8 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                             if constexpr (RECOMP) dq = sub2(dq, MD);
                             const f32x2 g = mul2(dy[q], wp[q]);
                             s1 = add2(s1, g);
-                            if constexpr (FUSE_VAR) {
-                                sq = fma2(dq, dq, sq);
-                                s2 = fma2(g, dq, s2);             // sum g * d
-                            } else {
-                                const f32x2 xh = mul2(dq, Sx);
-                                s2 = fma2(g, xh, s2);             // sum g * xhat
-                            }
+                            if constexpr (FUSE_VAR) sq = fma2(dq, dq, sq);
+                            s2 = fma2(g, dq, s2);                 // sum g * d
                         }
                     }
                 }
@@ -532,10 +530,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                 abort = group_exchange<W>(a, b, abort, slot, group, sub, lane);
             }
             const float na = -s * (a * inv_C);
-            // b is the sum of g * d (d = x - mean), or of g * xhat when
-            // pass 1 already knew rstd and did not keep d
-            constexpr bool B_OF_D = KEEP_D || FUSE_VAR;
-            const float nc = B_OF_D ? -(s * s) * (s * (b * inv_C)) : -s * (b * inv_C);
+            const float nc = -(s * s) * (s * (b * inv_C));   // b: sum of g * d
             const f32x2 NA = pair(na, na);
             const f32x2 NCc = pair(nc, nc);
 #pragma unroll
@@ -562,10 +557,7 @@ ln_bwd_tma_kernel(T *__restrict__ dinp, float *__restrict__ partial,
                                 f32x2 dq = sub2(pair_at<T>(xv[i], q), K);
                                 if constexpr (RECOMP) dq = sub2(dq, MD);
                                 xh = mul2(dq, Sx);
-                                if constexpr (FUSE_VAR)
-                                    o[q] = fma2(g, Sx, fma2(dq, NCc, NA));
-                                else
-                                    o[q] = fma2(g, Sx, fma2(xh, NCc, NA));
+                                o[q] = fma2(g, Sx, fma2(dq, NCc, NA));
                             }
                             acc_w[i][q] = fma2(dy, xh, acc_w[i][q]);
                             acc_b[i][q] = add2(acc_b[i][q], dy);
