@@ -35,6 +35,10 @@
  * Semantics shared by every call.
  *   - Asynchronous on `stream` (NULL: the legacy default stream); no host
  *     synchronisation; the library creates no streams of its own.
+ *   - Any number of host threads may call at once, each on its own stream:
+ *     the library's per-device state and caches are guarded, and results do
+ *     not depend on which thread called first (ln_backward_noalloc's shared
+ *     array is the one exception; see there).
  *   - Outputs are overwritten, never accumulated into, except where
  *     ln_backward_ex is asked to accumulate.
  *   - Results are deterministic: the same inputs give bitwise-identical

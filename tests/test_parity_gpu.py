@@ -548,3 +548,26 @@ def test_aliased_outputs_refused(lib):
         lib.ln_backward(y, dw, dw, x, x.clone(), w, m, r, N, C, lib.LN_BF16)
     assert e.value.status == lib.LN_ERR_ALIAS
     assert lib.launch_count() == n0
+
+
+def test_concurrent_host_threads(lib):
+    """Several host threads call the library at once, on their own streams,
+    as the first calls of a fresh process (so the per-device set-up, the
+    kernels' shared-memory limits and the occupancy cache fill concurrently),
+    on widths that reach the one-warp, two-warp, shared-row, split and fp32
+    kernels.  Every output equals the same calls made afterwards from one
+    thread, bit for bit; no call fails; no bounded wait ran out."""
+    import json
+    import os
+    import subprocess
+    import sys
+    script = os.path.join(os.path.dirname(os.path.abspath(__file__)), "threads_check.py")
+    proc = subprocess.run([sys.executable, script], capture_output=True, text=True,
+                          timeout=600)
+    assert proc.returncode == 0, proc.stderr[-3000:]
+    res = json.loads([l for l in proc.stdout.splitlines() if l.startswith("{")][-1])
+    assert res["errors"] == [], res["errors"]
+    assert res["mismatches"] == [], res["mismatches"]
+    assert res["device_status"] == 0
+    # per thread and round: forward 1 launch, each backward 2
+    assert res["threaded_launches"] == 6 * 12 * 5
