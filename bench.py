@@ -562,12 +562,13 @@ def run_workloads(torch, ln, stream, dev, nsets: int, calls: int = LOOP_CALLS) -
     like the headline: `calls` back-to-back calls over rotating buffer sets
     (a backward reads a set whose forward ran ``nsets // 2`` calls earlier),
     CUDA events around the loop on the launching stream.  ``fwd_us`` and
-    ``bwd_us`` time loops of one call kind; ``step_us`` times the step itself,
-    forward and backward alternating as in the headline's timed region, and
-    ``GB_s``, ``frac`` and ``rows_per_s`` come from it.  ``graph_step_us`` is
-    the same step loop captured in one CUDA graph and replayed (the library's
+    ``bwd_us`` time loops of one call kind, and ``GB_s``, ``frac`` and
+    ``rows_per_s`` are fwd+bwd as bytes / (t_fwd + t_bwd).  ``step_us`` times
+    the step itself, forward and backward alternating as in the headline's
+    timed region (``step_GB_s``, ``step_frac``); ``graph_step_us`` is the
+    same step loop captured in one CUDA graph and replayed (the library's
     calls are capturable), which removes the host's launch path but not the
-    kernels' own boundaries.  GB/s counts compulsory bytes; ``frac`` is
+    kernels' own boundaries.  GB/s counts compulsory bytes; fractions are
     against the measured HBM copy bandwidth (or the fallback, as
     ``peak_kind`` says)."""
     import numpy as np
@@ -630,18 +631,21 @@ def run_workloads(torch, ln, stream, dev, nsets: int, calls: int = LOOP_CALLS) -
         s_us = call_loop_us(torch, stream, step, calls)
         g_us = graph_loop_us(torch, stream, step)
         fb, bb = w.fwd_bytes(), w.bwd_bytes()
+        sum_gbs = (fb + bb) / ((f_us + b_us) * 1e-6) / 1e9
         step_gbs = (fb + bb) / (s_us * 1e-6) / 1e9
         graph_gbs = (fb + bb) / (g_us * 1e-6) / 1e9
         out[name] = {
             "N": N, "C": C, "dtype": w.dtype,
             "fwd_us": round(f_us, 3), "bwd_us": round(b_us, 3),
-            "step_us": round(s_us, 3), "graph_step_us": round(g_us, 3),
             "fwd_GB_s": round(fb / (f_us * 1e-6) / 1e9, 1),
             "bwd_GB_s": round(bb / (b_us * 1e-6) / 1e9, 1),
-            "GB_s": round(step_gbs, 1), "rows_per_s": round(N / (s_us * 1e-6), 1),
-            "frac": round(step_gbs / peak, 4),
+            "GB_s": round(sum_gbs, 1), "rows_per_s": round(N / ((f_us + b_us) * 1e-6), 1),
+            "frac": round(sum_gbs / peak, 4),
             "bwd_frac": round(bb / (b_us * 1e-6) / 1e9 / peak, 4),
-            "graph_GB_s": round(graph_gbs, 1), "graph_frac": round(graph_gbs / peak, 4),
+            "step_us": round(s_us, 3), "step_GB_s": round(step_gbs, 1),
+            "step_frac": round(step_gbs / peak, 4),
+            "graph_step_us": round(g_us, 3), "graph_GB_s": round(graph_gbs, 1),
+            "graph_frac": round(graph_gbs / peak, 4),
             "bytes": fb + bb,
             "l2": ("inputs smaller than L2: launch-bound correctness case"
                    if nsets * 2 * N * C * w.elem_bytes < 126e6 else
