@@ -1,6 +1,6 @@
 """The benchmark's multi-rank host logic on CPU: two gloo ranks (no GPU).
 
-On a GPU machine bench.py runs one rank per GPU over NCCL; the parts that decide
+On a multi-GPU node bench.py runs one rank per GPU over NCCL; the parts that decide
 the reported number -- the max over ranks of every timing, the whole-job
 throughput, and which rank prints -- do not depend on the backend and are
 exercised here with gloo."""
