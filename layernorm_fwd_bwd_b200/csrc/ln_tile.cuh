@@ -59,9 +59,17 @@ __device__ __forceinline__ bool tile_wait(uint64_t *bar, unsigned *status, unsig
 // Resident blocks per SM the register allocation must allow.  Wide 16-bit
 // rows on one warp (6+ vectors per lane, 2.4+ KB) fit three 2-tile blocks of
 // 8 warps in shared memory; unconstrained they take 82+ registers and only
-// two blocks would fit.  (0: no constraint.)
+// two blocks would fit.  fp32 rows of 5-8 vectors per lane: unconstrained,
+// ptxas settles at 48 registers and spills; a bound of three blocks gives it
+// 74-80 registers without spills, at 5-6 vectors one resident block fewer
+// than shared memory would allow (measured on B200: fp32 C = 768 62.1 ->
+// 61.4 us, C = 896 42.6 -> 42.2, C = 640 and 1024 unchanged).  (0: no
+// constraint.)
 #ifndef LN_TILE_FWD_MINB
-#define LN_TILE_FWD_MINB(T, V, NW) (((NW) == 8 && sizeof(T) == 2 && (V) >= 6) ? 3 : 0)
+#define LN_TILE_FWD_MINB(T, V, NW)                                                 \
+    (((NW) == 8 && ((sizeof(T) == 2 && (V) >= 6) || (sizeof(T) == 4 && (V) >= 5))) \
+         ? 3                                                                       \
+         : 0)
 #endif
 // Requirements (checked by the host): inp/out/weight/bias (and branch,
 // resid_out) 16-byte aligned, C * sizeof(T) a multiple of 16,
